@@ -1,0 +1,134 @@
+"""Gated Delta Rule-2 oracle (fp64, CPU) -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package. The CUDA library never calls it and shares no
+code with it.
+
+The arithmetic lives in ``gdr2_oracle.c`` (plain sequential fp64 C, one token
+at a time); this module compiles it with gcc on first use and wraps it for
+numpy arrays. Every input is upcast to float64 before the call, so bf16 inputs
+enter the oracle with exactly the values the GPU sees.
+
+Pinned by: tests/test_oracle_pins.py (KDA and Gated DeltaNet reductions,
+exact recall, b=0 closed form, brute-force transition products, the
+fast-weight argmin identity, state passing, varlen splitting, linearity).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr2_oracle.c")
+_LIB = os.path.join(_HERE, "libgdr2_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libgdr2_oracle.so`` (gcc, -O2, OpenMP)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c99",
+           "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.gdr2_oracle_forward.restype = ctypes.c_int
+            lib.gdr2_oracle_forward.argtypes = [
+                _D, _D, _D, _D, _D, _D, _D, _I64,
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                ctypes.c_int64, ctypes.c_int64, _D, _D, ctypes.c_int]
+            lib.gdr2_oracle_step.restype = ctypes.c_int
+            lib.gdr2_oracle_step.argtypes = [
+                _D, _D, _D, _D, _D, _D, _D,
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                _D, ctypes.c_int]
+            lib.gdr2_oracle_max_threads.restype = ctypes.c_int
+            lib.gdr2_oracle_max_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a):
+    return a.ctypes.data_as(_D) if a is not None else None
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP loop uses by default on this host."""
+    return int(_load().gdr2_oracle_max_threads())
+
+
+def forward(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None,
+            num_threads: int = 0):
+    """Token-by-token fp64 forward of Gated Delta Rule-2.
+
+    q, k, log_alpha, b: [B, T, H, d_k]; v, w: [B, T, H, d_v] (any float dtype,
+    upcast to fp64). init_state: [N, H, d_k, d_v] or None (zeros).
+    cu_seqlens: int array of N+1 offsets (then B must be 1) or None (N = B).
+    Returns (o [B, T, H, d_v], final_state [N, H, d_k, d_v]) as float64.
+    """
+    q, k, v, la, b, w = (_f64(x) for x in (q, k, v, log_alpha, b, w))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, x, d in (("k", k, dk), ("log_alpha", la, dk), ("b", b, dk),
+                       ("v", v, dv), ("w", w, dv)):
+        if x.shape != (B, T, H, d):
+            raise ValueError(f"{name} has shape {x.shape}, expected {(B, T, H, d)}")
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        cu = None
+        N = B
+    s0 = _f64(init_state) if init_state is not None else None
+    if s0 is not None and s0.shape != (N, H, dk, dv):
+        raise ValueError(f"init_state has shape {s0.shape}, expected {(N, H, dk, dv)}")
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().gdr2_oracle_forward(
+        _p(q), _p(k), _p(v), _p(la), _p(b), _p(w), _p(s0),
+        cu.ctypes.data_as(_I64) if cu is not None else None,
+        B, T, H, dk, dv, N, _p(o), _p(sf), int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle forward rejected its arguments (code {rc})")
+    return o, sf
+
+
+def step(q, k, v, log_alpha, b, w, state, num_threads: int = 0):
+    """One fp64 decode step. Token tensors [N, H, d]; state [N, H, d_k, d_v].
+
+    Returns (o [N, H, d_v], new_state) without modifying the caller's array.
+    """
+    q, k, v, la, b, w = (_f64(x) for x in (q, k, v, log_alpha, b, w))
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    S = np.array(state, dtype=np.float64, order="C", copy=True)
+    if S.shape != (N, H, dk, dv):
+        raise ValueError(f"state has shape {S.shape}, expected {(N, H, dk, dv)}")
+    o = np.zeros((N, H, dv), dtype=np.float64)
+    rc = _load().gdr2_oracle_step(_p(q), _p(k), _p(v), _p(la), _p(b), _p(w),
+                                  _p(S), N, H, dk, dv, _p(o), int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle step rejected its arguments (code {rc})")
+    return o, S

@@ -1,0 +1,140 @@
+"""Pin the fp64 oracle to what the pages fix, and show the pins have teeth.
+
+The first group runs every check in ``pins.py`` against the compiled oracle.
+The second group plants one plausible mistake at a time in a small
+pure-Python copy of the token loop (CPU only) and asserts that at least one
+pin rejects it, while the unmutated copy passes them all.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import pins
+
+
+def oracle_fwd(q, k, v, la, b, w, s0=None, cu=None):
+    return oracle.forward(q, k, v, la, b, w, s0, cu)
+
+
+def oracle_step(q, k, v, la, b, w, s):
+    return oracle.step(q, k, v, la, b, w, s)
+
+
+@pytest.mark.parametrize("pin", pins.FORWARD_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin(oracle_fwd, np.random.default_rng(1234))
+
+
+def test_oracle_fast_weight_argmin():
+    pins.pin_fast_weight_argmin(oracle_step, np.random.default_rng(7))
+
+
+def test_oracle_step_matches_single_token_forward():
+    rng = np.random.default_rng(3)
+    q, k, v, la, b, w, s0 = pins.rand_problem(rng, T=1)
+    o_f, s_f = oracle.forward(q, k, v, la, b, w, s0)
+    sq = lambda x: x[:, 0]
+    o_s, s_s = oracle.step(sq(q), sq(k), sq(v), sq(la), sq(b), sq(w), s0)
+    assert np.array_equal(o_f[:, 0], o_s) and np.array_equal(s_f, s_s)
+
+
+def test_oracle_zero_length_and_rejects_bad_args():
+    rng = np.random.default_rng(5)
+    q, k, v, la, b, w, s0 = pins.rand_problem(rng, T=0)
+    o, sf = oracle.forward(q, k, v, la, b, w, s0)
+    assert o.shape == (2, 0, 2, 5) and np.array_equal(sf, s0)
+    q, k, v, la, b, w, _ = pins.rand_problem(rng, B=1, T=4)
+    with pytest.raises(ValueError):
+        oracle.forward(q, k, v, la, b, w, None, np.array([0, 3, 2, 4]))
+    with pytest.raises(ValueError):
+        oracle.forward(q, k, v, la, b, w, None, np.array([0, 2, 3]))
+
+
+def test_oracle_threads_do_not_change_results():
+    rng = np.random.default_rng(11)
+    q, k, v, la, b, w, s0 = pins.rand_problem(rng, B=3, T=20, H=3)
+    o1, s1 = oracle.forward(q, k, v, la, b, w, s0, num_threads=1)
+    o4, s4 = oracle.forward(q, k, v, la, b, w, s0, num_threads=4)
+    assert np.array_equal(o1, o4) and np.array_equal(s1, s4)
+
+
+# --------------------------------------------------------------------------
+# Mutation tests: a small pure-Python token loop with one planted mistake.
+# --------------------------------------------------------------------------
+def loop_forward(q, k, v, la, b, w, s0=None, cu=None, mutation=None):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu is None:
+        spans = [(n, n * T, n * T + T) for n in range(B)]
+        flat = lambda x: x.reshape(B * T, H, x.shape[-1])
+    else:
+        spans = [(n, int(cu[n]), int(cu[n + 1])) for n in range(len(cu) - 1)]
+        flat = lambda x: x.reshape(T, H, x.shape[-1])
+    qf, kf, vf, laf, bf, wf = (flat(x) for x in (q, k, v, la, b, w))
+    o = np.zeros((qf.shape[0], H, dv))
+    sf = np.zeros((len(spans), H, dk, dv))
+    for n, t0, t1 in spans:
+        for h in range(H):
+            S = s0[n, h].copy() if s0 is not None else np.zeros((dk, dv))
+            for t in range(t0, t1):
+                kt, qt, bt = kf[t, h], qf[t, h], bf[t, h]
+                a = np.exp(laf[t, h])
+                e = bt * kt
+                z = wf[t, h] * vf[t, h]
+                if mutation == "drop_erase_gate":
+                    e = kt
+                if mutation == "drop_write_gate":
+                    z = vf[t, h]
+                if mutation == "readout_before_update":
+                    o[t, h] = S.T @ qt
+                if mutation != "decay_after_edit":
+                    S = a[:, None] * S
+                if mutation == "erase_gate_on_left":
+                    S = S + np.outer(bt * kt, z - kt @ S)
+                elif mutation == "wrong_sign":
+                    S = S + np.outer(kt, z + e @ S)
+                else:
+                    S = S + np.outer(kt, z - e @ S)
+                if mutation == "decay_after_edit":
+                    S = a[:, None] * S
+                if mutation == "decay_inverse":
+                    S = S / (a * a)[:, None]
+                if mutation != "readout_before_update":
+                    o[t, h] = S.T @ qt
+            sf[n, h] = S
+    return o.reshape(q.shape[:-1] + (dv,)), sf
+
+
+def loop_step(q, k, v, la, b, w, s, mutation=None):
+    ex = lambda x: x[:, None]
+    o, sf = loop_forward(ex(q), ex(k), ex(v), ex(la), ex(b), ex(w), s, mutation=mutation)
+    return o[:, 0], sf
+
+
+MUTATIONS = ["drop_erase_gate", "drop_write_gate", "readout_before_update",
+             "decay_after_edit", "erase_gate_on_left", "wrong_sign", "decay_inverse"]
+
+
+def _run_all_pins(fwd, step):
+    failures = []
+    for pin in pins.FORWARD_PINS:
+        try:
+            pin(fwd, np.random.default_rng(99))
+        except AssertionError as e:
+            failures.append(f"{pin.__name__}: {e}")
+    try:
+        pins.pin_fast_weight_argmin(step, np.random.default_rng(98))
+    except AssertionError as e:
+        failures.append(f"argmin: {e}")
+    return failures
+
+
+def test_unmutated_loop_passes_every_pin():
+    assert _run_all_pins(loop_forward, loop_step) == []
+
+
+@pytest.mark.parametrize("mutation", MUTATIONS)
+def test_planted_mistake_is_caught(mutation):
+    fwd = lambda *a, **kw: loop_forward(*a, mutation=mutation, **kw)
+    step = lambda *a, **kw: loop_step(*a, mutation=mutation, **kw)
+    assert _run_all_pins(fwd, step), f"no pin caught mutation {mutation!r}"

@@ -1,0 +1,161 @@
+/*
+ * gdr2.h -- C ABI of the B200 (sm_100a) Gated Delta Rule-2 operator library.
+ *
+ * The operator (Gated DeltaNet-2's sequence mixer). Per sequence and head the
+ * recurrent state S is a d_k x d_v matrix and each token t updates it as
+ *
+ *     S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T,
+ *     o_t = S_t^T q_t,                       alpha_t = exp(log_alpha_t),
+ *
+ * where "." is the element-wise product, b_t in [0,1]^{d_k} is the erase gate
+ * (key side) and w_t in [0,1]^{d_v} the write gate (value side). Sources:
+ *   - "Gated DeltaNet-2: Decoupling Erase and Write Gates in Linear Attention
+ *     for Better Memory Editing" (zhichai.net), section "Gated Delta Rule-2":
+ *     the update rule and the two gates;
+ *   - "엔비디아, 기억 수정 최적화 선형 어텐션 모델 공개" (ainews.random.gg),
+ *     section "Gated Delta Rule-2: two gates instead of one": D_t =
+ *     Diag(alpha_t) is channel-wise over key channels and the decay comes
+ *     before the active edit; section "Chunkwise training and gate-aware
+ *     backward": the chunkwise WY form with the cumulative channel-wise decay
+ *     absorbed into asymmetric erase factors I - kbar_r ebar_r^T, chunk size
+ *     C = 64;
+ *   - same article, lead paragraph: decoding runs the recurrence one token at
+ *     a time in constant memory.
+ * The readout uses the post-update state; q is not scaled; the gates arrive
+ * already in [0,1] and log_alpha already in log space (nothing is activated
+ * or normalised inside the operator).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     and 16-byte aligned. The library never allocates, frees or synchronises;
+ *     every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and runs on the device that is current on the calling
+ *     thread.
+ *   - Token tensors are token-major: q, k, b, log_alpha are [B, T, H, d_k];
+ *     v, w, o are [B, T, H, d_v]. States are [N, H, d_k, d_v] fp32 with d_v
+ *     contiguous (row c of a head's state is key channel c).
+ *   - q, k, v, b, w and o share `dtype`; log_alpha and states are always fp32.
+ *   - Supported shapes: d_k = d_v in {64, 128}; H >= 1; sizes below 2^31
+ *     elements per tensor.
+ *   - Host-side validation happens before any launch; on failure nothing is
+ *     launched and the status says why. A launch failure returns
+ *     GDR2_ERR_CUDA (the CUDA error is then also pending in the runtime).
+ *     Errors raised while kernels run surface at the caller's next
+ *     synchronisation, as for any CUDA kernel.
+ *   - `o` may not alias any input. Calls that share output or state buffers
+ *     must be ordered by the caller (same stream or events).
+ *   - Decay range: within one 64-token chunk the summed log_alpha of any key
+ *     channel must stay above -80 (per-token alpha above ~0.29 on average);
+ *     below that the chunk form's fp32 decay factors leave the fp32 range.
+ */
+#ifndef GDR2_H_
+#define GDR2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR2_OK = 0,
+    GDR2_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, bad dtype */
+    GDR2_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d_k != d_v) */
+    GDR2_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    GDR2_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    GDR2_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait gave up */
+} gdr2_status;
+
+typedef enum {
+    GDR2_FP32 = 0,
+    GDR2_BF16 = 1
+} gdr2_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gdr2_status_string(gdr2_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int gdr2_version(void);
+
+/*
+ * gdr2_chunk_fwd -- chunkwise-parallel forward (prefill / training forward).
+ *
+ * Computes o_t for every token and the state after the last token of every
+ * sequence, with the chunk form of the recurrence (C = 64): inside a chunk
+ * the cumulative log-decay g_r (relative to the chunk start, fp32) turns the
+ * token transitions into asymmetric rank-one factors I - kbar_r ebar_r^T with
+ * kbar_r = k_r . exp(-g_r) and ebar_r = b_r . k_r . exp(g_r); the strictly
+ * lower 64 x 64 matrix A = tril(Ebar Kbar^T) gives T = (I + A)^{-1}, the WY
+ * factors W = T Ebar and U = T Z - W S0 (Z = W_gate . V), and then
+ *     O   = Qbar S0 + tril(Qbar Kbar^T) U,        Qbar = Q . exp(g),
+ *     S_C = Diag(exp(g_C)) S0 + (K . exp(g_C - g))^T U.
+ * ("Chunkwise training and gate-aware backward", ainews.random.gg article.)
+ *
+ * Arguments
+ *   q, k, b      [B, T, H, d_k] in `dtype`
+ *   v, w         [B, T, H, d_v] in `dtype`     (w is the write gate)
+ *   log_alpha    [B, T, H, d_k] fp32           (log of the per-channel decay)
+ *   init_state   [N, H, d_k, d_v] fp32, or NULL for zero initial states
+ *   cu_seqlens   NULL, or a DEVICE int32 array of N+1 offsets for a packed
+ *                variable-length batch: then B must be 1, sequence n covers
+ *                tokens cu_seqlens[n] .. cu_seqlens[n+1]-1, offsets must be
+ *                non-decreasing with cu_seqlens[0] = 0 and cu_seqlens[N] = T
+ *                (the device values are trusted; they are not read on the
+ *                host). Chunks restart at every sequence start.
+ *   B, T, H      batch, tokens per sequence (total tokens when packed), heads
+ *   d_k, d_v     key / value head dimensions
+ *   num_seqs     N: must equal B without cu_seqlens
+ *   dtype        GDR2_FP32 or GDR2_BF16 for q, k, v, b, w, o
+ *   o            [B, T, H, d_v] in `dtype` (output)
+ *   final_state  [N, H, d_k, d_v] fp32 (output), or NULL to skip it;
+ *                may alias init_state (each head reads its initial state
+ *                before it writes its final state)
+ *   workspace, workspace_bytes
+ *                device scratch of at least gdr2_chunk_fwd_workspace_size()
+ *                bytes (NULL allowed when that size is 0)
+ *   stream       cudaStream_t
+ * Precision: with GDR2_FP32 every product runs in fp32 on CUDA cores; with
+ * GDR2_BF16 the dense intra-chunk contractions run on the tensor cores with
+ * bf16 operands and fp32 accumulation while the state stays fp32.
+ */
+gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const void *b, const void *w,
+                           const float *init_state, const int32_t *cu_seqlens,
+                           int64_t B, int64_t T, int64_t H, int64_t d_k,
+                           int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                           void *o, float *final_state, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/* Scratch bytes gdr2_chunk_fwd needs for this problem (written to *bytes). */
+gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
+                                          int64_t d_k, int64_t d_v,
+                                          int64_t num_seqs, gdr2_dtype dtype,
+                                          size_t *bytes);
+
+/*
+ * gdr2_recurrent_step -- one decode step for N independent sequences.
+ *
+ * For every sequence n and head h, with the state updated IN PLACE:
+ *     S <- (I - k (b . k)^T) Diag(exp(log_alpha)) S + k (w . v)^T,
+ *     o  = S^T q.
+ * ("Gated Delta Rule-2" section of the zhichai.net summary; decoding to
+ * constant memory per the ainews.random.gg article's lead.)
+ *
+ *   q, k, b      [N, H, d_k] in `dtype`;  log_alpha [N, H, d_k] fp32
+ *   v, w         [N, H, d_v] in `dtype`
+ *   state        [N, H, d_k, d_v] fp32, read and written in place
+ *   o            [N, H, d_v] in `dtype` (output)
+ * No workspace. Each (n, h) is independent, so N may be any batch size.
+ */
+gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const void *b,
+                                const void *w, float *state, int64_t N,
+                                int64_t H, int64_t d_k, int64_t d_v,
+                                gdr2_dtype dtype, void *o, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR2_H_ */

@@ -1,0 +1,126 @@
+// C ABI of the Gated Delta Rule-2 library: argument validation and dispatch.
+// Declarations and the full contract are in include/gdr2.h.
+#include "../../include/gdr2.h"
+#include "kernels.h"
+
+#include <cuda_runtime.h>
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int64_t d) { return d == 64 || d == 128; }
+
+gdr2_status check_dims(int64_t d_k, int64_t d_v)
+{
+    if (d_k <= 0 || d_v <= 0) return GDR2_ERR_INVALID_ARG;
+    if (d_k != d_v || !supported_dim(d_k)) return GDR2_ERR_UNSUPPORTED;
+    return GDR2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdr2_status_string(gdr2_status s)
+{
+    switch (s) {
+    case GDR2_OK: return "ok";
+    case GDR2_ERR_INVALID_ARG: return "invalid argument";
+    case GDR2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GDR2_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDR2_ERR_CUDA: return "CUDA error";
+    case GDR2_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int gdr2_version(void) { return kVersion; }
+
+gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k,
+                                          int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                                          size_t *bytes)
+{
+    if (!bytes) return GDR2_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    *bytes = 0;
+    return GDR2_OK;
+}
+
+gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *init_state,
+                           const int32_t *cu_seqlens, int64_t B, int64_t T, int64_t H,
+                           int64_t d_k, int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                           void *o, float *final_state, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    if (cu_seqlens) {
+        if (B != 1) return GDR2_ERR_INVALID_ARG;
+    } else if (num_seqs != B) {
+        return GDR2_ERR_INVALID_ARG;
+    }
+    if (H > 65535 || num_seqs > 65535) return GDR2_ERR_UNSUPPORTED;
+    const int64_t tokens = B * T;
+    if (tokens > 0) {
+        const void *ptrs[] = {q, k, v, log_alpha, b, w, o};
+        for (const void *p : ptrs)
+            if (!p || !aligned16(p)) return GDR2_ERR_INVALID_ARG;
+    }
+    if (init_state && !aligned16(init_state)) return GDR2_ERR_INVALID_ARG;
+    if (final_state && !aligned16(final_state)) return GDR2_ERR_INVALID_ARG;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDR2_ERR_INVALID_ARG;
+    size_t need = 0;
+    st = gdr2_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, dtype, &need);
+    if (st != GDR2_OK) return st;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDR2_ERR_WORKSPACE;
+    if (num_seqs == 0) return GDR2_OK;
+
+    gdr2::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w;
+    a.log_alpha = log_alpha;
+    a.init_state = init_state;
+    a.cu_seqlens = cu_seqlens;
+    a.o = o;
+    a.final_state = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.num_seqs = num_seqs;
+    a.bf16 = dtype == GDR2_BF16;
+    cudaError_t e = gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const void *b, const void *w,
+                                float *state, int64_t N, int64_t H, int64_t d_k, int64_t d_v,
+                                gdr2_dtype dtype, void *o, void *stream)
+{
+    if (N < 0 || H <= 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    if (N * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;
+    if (N == 0) return GDR2_OK;
+    const void *ptrs[] = {q, k, v, log_alpha, b, w, state, o};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return GDR2_ERR_INVALID_ARG;
+
+    gdr2::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w;
+    a.log_alpha = log_alpha;
+    a.state = state;
+    a.o = o;
+    a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
+    a.bf16 = dtype == GDR2_BF16;
+    cudaError_t e = gdr2::launch_decode(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+}  // extern "C"

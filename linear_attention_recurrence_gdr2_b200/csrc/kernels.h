@@ -1,0 +1,34 @@
+// Internal launch interface between the C ABI (gdr2_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdr2 {
+
+struct DecodeArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *log_alpha;
+    float *state;
+    void *o;
+    int64_t N, H, dk, dv;
+    bool bf16;
+};
+
+struct ChunkArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *log_alpha;
+    const float *init_state;   // may be null
+    const int32_t *cu_seqlens; // may be null
+    void *o;
+    float *final_state;        // may be null
+    int64_t B, T, H, dk, dv, num_seqs;
+    bool bf16;
+};
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// fp32 CUDA-core chunk forward (any dtype; the fp32 path of the library).
+cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
+
+}  // namespace gdr2

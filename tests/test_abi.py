@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports what include/gdr2.h declares, and rejects
+bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_recurrence_gdr2_b200 as gdr2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(gdr2_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("gdr2_chunk_fwd", "gdr2_recurrent_step", "gdr2_chunk_fwd_workspace_size",
+               "gdr2_status_string", "gdr2_version"):
+        assert fn in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_library_exports_declared_symbol(name):
+    lib = ctypes.CDLL(gdr2.LIB_PATH)
+    assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings_and_version():
+    assert gdr2.status_string(0) == "ok"
+    for s in range(1, 6):
+        assert gdr2.status_string(s) not in ("ok", "unknown status")
+    assert gdr2.status_string(99) == "unknown status"
+    assert gdr2.version() >= 100
+
+
+def test_workspace_size_query():
+    assert gdr2.workspace_size(4, 2048, 16, 128, 128, 4, gdr2.GDR2_BF16) >= 0
+    with pytest.raises(gdr2.GDR2Error) as e:
+        gdr2.workspace_size(4, 2048, 16, 96, 96, 4, gdr2.GDR2_BF16)
+    assert e.value.status == UNSUPPORTED
+    with pytest.raises(gdr2.GDR2Error) as e:
+        gdr2.workspace_size(4, 2048, 0, 128, 128, 4, gdr2.GDR2_BF16)
+    assert e.value.status == INVALID
+
+
+def _chunk(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, s0=None, cu=None,
+             B=2, T=128, H=4, dk=128, dv=128, N=2, dtype=1, o=FAKE, sf=FAKE,
+             ws=None, wsb=0, stream=None)
+    a.update(over)
+    return gdr2.lib().gdr2_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["b"], a["w"], a["s0"],
+                                     a["cu"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"],
+                                     a["dtype"], a["o"], a["sf"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), INVALID),
+    (dict(o=None), INVALID),
+    (dict(la=FAKE + 4), INVALID),          # misaligned
+    (dict(v=FAKE + 2), INVALID),
+    (dict(H=0), INVALID),
+    (dict(T=-1), INVALID),
+    (dict(dtype=7), INVALID),
+    (dict(N=3), INVALID),                  # num_seqs != B without cu_seqlens
+    (dict(cu=FAKE, B=2), INVALID),         # packed batch needs B == 1
+    (dict(dk=96, dv=96), UNSUPPORTED),
+    (dict(dk=128, dv=64), UNSUPPORTED),
+    (dict(dk=0, dv=128), INVALID),
+    (dict(s0=FAKE + 8), INVALID),
+    (dict(sf=FAKE + 8), INVALID),
+    (dict(H=70000), UNSUPPORTED),
+])
+def test_chunk_fwd_rejects_bad_arguments(over, expect):
+    assert _chunk(**over) == expect
+
+
+def _step(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, s=FAKE, N=4, H=2, dk=64, dv=64,
+             dtype=0, o=FAKE, stream=None)
+    a.update(over)
+    return gdr2.lib().gdr2_recurrent_step(a["q"], a["k"], a["v"], a["la"], a["b"], a["w"],
+                                          a["s"], a["N"], a["H"], a["dk"], a["dv"], a["dtype"],
+                                          a["o"], a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(s=None), INVALID),
+    (dict(k=FAKE + 1), INVALID),
+    (dict(N=-1), INVALID),
+    (dict(H=0), INVALID),
+    (dict(dtype=3), INVALID),
+    (dict(dk=32, dv=32), UNSUPPORTED),
+])
+def test_recurrent_step_rejects_bad_arguments(over, expect):
+    assert _step(**over) == expect
+
+
+def test_empty_problems_return_ok_without_launch():
+    assert _chunk(B=0, N=0, q=None, o=None) == OK
+    assert _chunk(B=1, T=0, N=0, cu=FAKE) == OK
+    assert _step(N=0, q=None, s=None) == OK

@@ -1,0 +1,202 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small cases compare every element; the full-size workloads compare whole
+(sequence, head) units that the oracle recomputes one by one, in the same
+launch configuration the benchmark times. Bound: relative L2 error <= 1e-4
+for fp32 inputs and <= 5e-3 for bf16 inputs (fp32 state), on o and on the
+final state; the per-element max error is printed beside it.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import TOL, assert_close, rel_l2, to_np, unit_slices, upload
+from linear_attention_recurrence_gdr2_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+
+def gdr2():
+    import linear_attention_recurrence_gdr2_b200 as m
+    return m
+
+
+def run_chunk(inp, device, final=True):
+    t = upload(inp, device)
+    o, sf = gdr2().chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"],
+                             t["init_state"], t["cu_seqlens"], output_final_state=final)
+    import torch
+    torch.cuda.synchronize()
+    return to_np(o), (to_np(sf) if sf is not None else None)
+
+
+def check_full(inp, device, label):
+    o, sf = run_chunk(inp, device)
+    o_r, sf_r = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w,
+                               inp.init_state, inp.cu_seqlens)
+    assert_close(f"{label} o", o, o_r, inp.dtype)
+    assert_close(f"{label} state", sf, sf_r, inp.dtype)
+
+
+def check_units(inp, device, units, label):
+    o, sf = run_chunk(inp, device)
+    for n, h in units:
+        sl, rows, s0 = unit_slices(inp, n, h)
+        o_r, sf_r = oracle.forward(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha),
+                                   sl(inp.b), sl(inp.w), s0)
+        assert_close(f"{label} unit({n},{h}) o", o[rows], o_r[0, :, 0], inp.dtype)
+        assert_close(f"{label} unit({n},{h}) state", sf[n, h], sf_r[0, 0], inp.dtype)
+    return o, sf
+
+
+# ---------------------------------------------------------------- chunk fwd
+def test_tiny_fp32_workload(cuda_device):
+    """B=1, H=1, T=256, d=64, fp32, zero initial state, seed 0: every element."""
+    check_full(gen.tiny_fp32(), cuda_device, "tiny fp32")
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_chunk_small_shapes(cuda_device, T, d, dtype):
+    inp = gen.make_inputs(2, T, 3, d, d, dtype, seed=T * 7 + d, init_std=0.05)
+    check_full(inp, cuda_device, f"T={T} d={d} {dtype}")
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_chunk_varlen_small(cuda_device, d, dtype):
+    lengths = [1, 64, 0, 130, 63, 65, 7, 192]
+    inp = gen.make_inputs(1, 0, 2, d, d, dtype, seed=d, init_std=0.05, lengths=lengths)
+    check_full(inp, cuda_device, f"varlen d={d} {dtype}")
+
+
+def test_chunk_zero_initial_state_and_no_final_state(cuda_device):
+    inp = gen.make_inputs(1, 100, 2, 128, 128, "bf16", seed=3)
+    o, sf = run_chunk(inp, cuda_device, final=False)
+    assert sf is None
+    o_r, _ = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w)
+    assert_close("no-final o", o, o_r, "bf16")
+
+
+def test_chunk_final_state_may_alias_initial_state(cuda_device):
+    import torch
+    inp = gen.make_inputs(2, 130, 2, 64, 64, "fp32", seed=4, init_std=0.1)
+    t = upload(inp, cuda_device)
+    s = t["init_state"].clone()
+    o, sf = gdr2().chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], s,
+                             final_state=s)
+    torch.cuda.synchronize()
+    o_r, sf_r = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w, inp.init_state)
+    assert_close("alias o", to_np(o), o_r, "fp32")
+    assert_close("alias state", to_np(s), sf_r, "fp32")
+
+
+def test_chunk_empty_sequence_keeps_state(cuda_device):
+    inp = gen.make_inputs(1, 0, 2, 64, 64, "bf16", seed=5, init_std=0.1, lengths=[0, 0])
+    o, sf = run_chunk(inp, cuda_device)
+    assert o.shape[1] == 0
+    assert np.array_equal(sf, inp.init_state.astype(np.float64))
+
+
+def test_chunk_deterministic(cuda_device):
+    inp = gen.make_inputs(2, 300, 4, 128, 128, "bf16", seed=6, init_std=0.01)
+    o1, s1 = run_chunk(inp, cuda_device)
+    o2, s2 = run_chunk(inp, cuda_device)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+
+
+def test_chunk_strong_decay_in_range(cuda_device):
+    """Per-token log-decay down to about -1 (chunk sums near -64) stays finite
+    and accurate: the pairwise factors keep e^{g_r - g_s} <= 1."""
+    inp = gen.make_inputs(1, 256, 2, 128, 128, "bf16", seed=8, la_scale=1.2, init_std=0.01)
+    check_full(inp, cuda_device, "strong decay")
+
+
+@pytest.mark.slow
+def test_layer_prefill_full_size(cuda_device):
+    """B=4, H=16, T=2048, d=128, bf16: six (sequence, head) units recomputed."""
+    inp = gen.layer_prefill()
+    check_units(inp, cuda_device, [(0, 0), (1, 5), (2, 9), (3, 15), (0, 13), (3, 2)], "prefill")
+
+
+@pytest.mark.slow
+def test_long_context_full_size(cuda_device):
+    """B=1, H=16, T=32768, d=128, bf16, slow forgetting, nonzero initial state."""
+    inp = gen.long_context()
+    check_units(inp, cuda_device, [(0, 0), (0, 11)], "long")
+
+
+@pytest.mark.slow
+def test_varlen_packed_full_size(cuda_device):
+    """64 packed sequences, lengths in [128, 8192], H=16, bf16, per-sequence states."""
+    inp = gen.varlen_packed()
+    lengths = np.diff(inp.cu_seqlens)
+    picks = [int(np.argmax(lengths)), int(np.argmin(lengths)), 17, 40]
+    check_units(inp, cuda_device, [(n, (3 * n) % 16) for n in picks], "varlen")
+
+
+# ------------------------------------------------------------------- decode
+def run_decode(dec, device, steps):
+    import torch
+    dt = torch.bfloat16 if dec.dtype == "bf16" else torch.float32
+    t = lambda x, d: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=d)
+    state = t(dec.state, torch.float32)
+    outs = []
+    for s in range(steps):
+        o = gdr2().recurrent_step(t(dec.q[s], dt), t(dec.k[s], dt), t(dec.v[s], dt),
+                                  t(dec.log_alpha[s], torch.float32), t(dec.b[s], dt),
+                                  t(dec.w[s], dt), state)
+        outs.append(to_np(o))
+    torch.cuda.synchronize()
+    return np.stack(outs), to_np(state)
+
+
+def oracle_decode(dec, steps):
+    S = dec.state
+    outs = []
+    for s in range(steps):
+        o, S = oracle.step(dec.q[s], dec.k[s], dec.v[s], dec.log_alpha[s], dec.b[s], dec.w[s], S)
+        outs.append(o)
+    return np.stack(outs), S
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_small(cuda_device, d, dtype):
+    dec = gen.make_decode_inputs(3, 5, d, d, 6, dtype, seed=d + 1)
+    o, S = run_decode(dec, cuda_device, 6)
+    o_r, S_r = oracle_decode(dec, 6)
+    for s in range(6):
+        assert_close(f"decode step {s} o", o[s], o_r[s], dtype)
+    assert_close("decode state", S, S_r, dtype)
+
+
+@pytest.mark.slow
+def test_decode_full_size(cuda_device):
+    """N=256 x H=16, d=128, fp32 state, 64 consecutive bf16 steps; all heads."""
+    dec = gen.decode_batch()
+    o, S = run_decode(dec, cuda_device, 64)
+    o_r, S_r = oracle_decode(dec, 64)
+    worst = max(rel_l2(o[s], o_r[s]) for s in range(64))
+    print(f"decode full: worst per-step o rel_l2 {worst:.3e}")
+    assert worst <= TOL["bf16"]
+    assert_close("decode full state", S, S_r, "bf16")
+
+
+def test_decode_matches_chunk_forward(cuda_device):
+    """T decode steps from S0 and one chunk_fwd over the same T tokens agree."""
+    import torch
+    inp = gen.make_inputs(2, 70, 3, 128, 128, "fp32", seed=9, init_std=0.05)
+    o_c, s_c = run_chunk(inp, cuda_device)
+    t = upload(inp, cuda_device)
+    state = t["init_state"].clone()
+    o_d = []
+    for s in range(70):
+        sl = lambda x: x[:, s].contiguous()
+        o_d.append(to_np(gdr2().recurrent_step(sl(t["q"]), sl(t["k"]), sl(t["v"]),
+                                               sl(t["log_alpha"]), sl(t["b"]), sl(t["w"]),
+                                               state)))
+    torch.cuda.synchronize()
+    assert rel_l2(np.stack(o_d, axis=1), o_c) < 1e-4
+    assert rel_l2(to_np(state), s_c) < 1e-4

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                 _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
                 _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            L.gdr2_check_device_error.restype = ctypes.c_int
+            L.gdr2_check_device_error.argtypes = [_vp]
             L.gdr2_recurrent_step.restype = ctypes.c_int
             L.gdr2_recurrent_step.argtypes = [
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -77,6 +79,14 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return int(lib().gdr2_version())
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronise `stream` and raise GDR2Error if a kernel of the library gave
+    up a bounded device-side wait since the last check (gdr2_check_device_error)."""
+    st = lib().gdr2_check_device_error(_stream_handle(stream))
+    if st != GDR2_OK:
+        raise GDR2Error("gdr2_check_device_error", st)
 
 
 def _dtype_code(t) -> int:

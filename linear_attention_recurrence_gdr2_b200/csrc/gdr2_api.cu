@@ -93,7 +93,8 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.num_seqs = num_seqs;
     a.bf16 = dtype == GDR2_BF16;
-    cudaError_t e = gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
+    cudaError_t e = gdr2::chunk_tc_supported(a) ? gdr2::launch_chunk_tc(a, (cudaStream_t)stream)
+                                                : gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
@@ -121,6 +122,14 @@ gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
     a.bf16 = dtype == GDR2_BF16;
     cudaError_t e = gdr2::launch_decode(a, (cudaStream_t)stream);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+gdr2_status gdr2_check_device_error(void *stream)
+{
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDR2_ERR_CUDA;
+    int code = 0;
+    if (gdr2::chunk_tc_read_and_clear_error(&code) != cudaSuccess) return GDR2_ERR_CUDA;
+    return code ? GDR2_ERR_DEVICE_TIMEOUT : GDR2_OK;
 }
 
 }  // extern "C"

@@ -31,4 +31,11 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // fp32 CUDA-core chunk forward (any dtype; the fp32 path of the library).
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 
+// Tensor-core chunk forward (bf16, d_k = d_v = 128).
+bool chunk_tc_supported(const ChunkArgs &a);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+
+// Reads and clears the tensor-core kernel's device error word (synchronous).
+cudaError_t chunk_tc_read_and_clear_error(int *code);
+
 }  // namespace gdr2

@@ -27,6 +27,7 @@ def run_chunk(inp, device, final=True):
                              t["init_state"], t["cu_seqlens"], output_final_state=final)
     import torch
     torch.cuda.synchronize()
+    gdr2().check_device_error()
     return to_np(o), (to_np(sf) if sf is not None else None)
 
 

@@ -30,10 +30,10 @@
 //
 // Warp roles (12 warps):
 //   0      TMA producer of q, k, b tiles (double-buffered slots)
-//   1      tcgen05.mma issuer (one thread, polls both pipelines)
+//   1      tcgen05.mma issuer of the prep pipeline ([A;P], W^T, U0^T)
 //   2      TMEM allocator; TMA producer of v tiles and L2 prefetch of
 //          log_alpha and w
-//   3      idle
+//   3      tcgen05.mma issuer of the state chain (U^T, O^T, state update)
 //   4..7   prep: cumulative decay, factors, Z, (I + A)^{-1}, W^T to smem
 //   8..11  epilogue: U^T to bf16, o stores, state scaling, final state
 // Every wait is bounded: after about a second without progress the CTA
@@ -48,6 +48,20 @@
 namespace gdr2 {
 
 __device__ int g_chunk_tc_error;
+
+// Optional per-phase SM-clock timestamps for the first CTAs (compiled in only
+// with -DGDR2_TRACE; the tracing driver points g_chunk_tc_trace at a buffer
+// of [4 CTAs][1024 chunks][32 events] uint64).
+#ifdef GDR2_TRACE
+__device__ unsigned long long *g_chunk_tc_trace;
+#define GDR2_TRACE_AT(chunk, ev)                                                           \
+    do {                                                                                   \
+        if (blockIdx.x < 4 && g_chunk_tc_trace && (chunk) < 1024)                          \
+            g_chunk_tc_trace[((size_t)blockIdx.x * 1024 + (chunk)) * 32 + (ev)] = clock64(); \
+    } while (0)
+#else
+#define GDR2_TRACE_AT(chunk, ev) do { } while (0)
+#endif
 
 namespace {
 
@@ -68,11 +82,13 @@ constexpr uint32_t kPB0 = 122880;        // P bf16, 64 rows x 128 B
 constexpr uint32_t kPB1 = 131072;
 constexpr uint32_t kWB0 = 139264;        // W^T bf16, 128 rows x 128 B
 constexpr uint32_t kWB1 = 155648;
-constexpr uint32_t kSA = 172032;         // fp32 A, 64 x 65
-constexpr uint32_t kST = kSA + 64 * 65 * 4;  // fp32 T, 64 x 65
-constexpr uint32_t kVEC = kST + 64 * 65 * 4; // half sums: T0[4][128], T1[4][128], f[128]
-constexpr uint32_t kBAR = kVEC + (8 * 128 + 128) * 4;
-constexpr int kNumBars = 20;
+constexpr int kLD = 68;                  // fp32 scratch row pitch (16-byte aligned rows)
+constexpr uint32_t kSA = 172032;         // fp32 A^T, 64 x kLD
+constexpr uint32_t kST = kSA + 64 * kLD * 4;  // fp32 T, 64 x kLD
+constexpr uint32_t kVEC = kST + 64 * kLD * 4; // half sums: T0[4][128], T1[4][128], f[128]
+constexpr uint32_t kBSUM = kVEC + (8 * 128 + 128) * 4;  // per-row-block log-decay sums [4][128]
+constexpr uint32_t kBAR = kBSUM + 4 * 128 * 4;
+constexpr int kNumBars = 23;
 constexpr uint32_t kMISC = kBAR + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kMISC + 64 + 1024;  // + alignment slack
 
@@ -80,7 +96,7 @@ constexpr uint32_t kSmemBytes = kMISC + 64 + 1024;  // + alignment slack
 enum {
     B_FULL0 = 0, B_FULL1, B_SLOTFREE0, B_SLOTFREE1, B_VFULL, B_VFREE, B_PREP, B_AP, B_T,
     B_WDONE, B_WREADY0, B_WREADY1, B_SREADY, B_UDONE, B_UCONV, B_SDONE, B_VEC0, B_VEC1,
-    B_DRAIN, B_SPARE
+    B_DRAIN, B_DRAIN2, B_UFREE0, B_UFREE1, B_LAFULL
 };
 
 // ---- TMEM column map ------------------------------------------------------
@@ -124,32 +140,85 @@ __device__ __forceinline__ bool group_and(uint32_t id, bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d) : "memory");
+// Bounded spin on a barrier phase without suspending (for the MMA issuers,
+// whose reaction time is on the chunk-to-chunk path).
+__device__ __forceinline__ bool spin_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         int site) {
+    uint64_t deadline = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 1023u) == 1023u) {
+            if (*abort_flag) return false;
+            const uint64_t now = globaltimer_ns();
+            if (deadline == 0) deadline = now + kWaitNs;
+            else if (now > deadline) {
+                *abort_flag = 1;
+                atomicCAS(&g_chunk_tc_error, 0, 0x100 | site);
+                return false;
+            }
+        }
+    }
 }
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
-__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// Warp-level D (16x8, fp32) += A (16x8, tf32) * B (8x8, tf32).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// One 16x8 output tile of C = X * Y over K (multiple of 8) on the tensor
+// cores in tf32 with fp32 accumulation; X(i, k) and Y(k, j) are fp32 values in
+// shared memory addressed as x[i * xsi + k * xsk] and y[k * ysk + j].
+template <int K>
+__device__ __forceinline__ void tile_tf32(float (&d)[4], const float *x, int xsi, int xsk,
+                                          const float *y, int ysk, int lane) {
+    const int ar = lane >> 2, ac = lane & 3;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t a[4], b[2];
+        a[0] = to_tf32(x[ar * xsi + (k0 + ac) * xsk]);
+        a[1] = to_tf32(x[(ar + 8) * xsi + (k0 + ac) * xsk]);
+        a[2] = to_tf32(x[ar * xsi + (k0 + ac + 4) * xsk]);
+        a[3] = to_tf32(x[(ar + 8) * xsi + (k0 + ac + 4) * xsk]);
+        b[0] = to_tf32(y[(k0 + ac) * ysk + ar]);
+        b[1] = to_tf32(y[(k0 + ac + 4) * ysk + ar]);
+        mma_tf32_16x8x8(d, a, b);
+    }
+}
+// Stores a 16x8 fp32 tile (times `scale`) at out[i * osi + j].
+__device__ __forceinline__ void store_tile(const float (&d)[4], float *out, int osi, int lane,
+                                           float scale) {
+    const int r = lane >> 2, c2 = 2 * (lane & 3);
+    *reinterpret_cast<float2 *>(out + r * osi + c2) = make_float2(scale * d[0], scale * d[1]);
+    *reinterpret_cast<float2 *>(out + (r + 8) * osi + c2) = make_float2(scale * d[2], scale * d[3]);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&v));
 }
 
 // Writes 64 fp32 values as one 128-byte bf16 row of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row_bf16_sw128(uint32_t tile, uint32_t row, const float *x) {
+__device__ __forceinline__ void store_row_bf16_sw128(unsigned char *tile, uint32_t row, const float *x) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        const uint32_t a = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
-        const uint32_t b = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
-        const uint32_t c = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
-        const uint32_t d = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
-        st_shared_v4(tile + sw128_offset(row, 16 * q), a, b, c, d);
+        uint4 u;
+        u.x = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
+        u.y = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
+        u.z = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
+        u.w = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
+        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, 16 * q)) = u;
     }
 }
 
@@ -160,8 +229,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 TcParams prm)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // Align to 1024 B by offsetting the __shared__ array itself (not through an
+    // integer round trip), so every access below stays a shared-space access.
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMISC);
@@ -171,6 +241,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     float *vecT0 = reinterpret_cast<float *>(smem + kVEC);         // [4][128]
     float *vecT1 = vecT0 + 4 * 128;                                 // [4][128]
     float *vecF = vecT1 + 4 * 128;                                  // [128]
+    float *vecBS = reinterpret_cast<float *>(smem + kBSUM);         // [4][128]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = prm.H;
@@ -223,6 +294,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 if (c >= 2 && !wait_bar(&bars[B_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, 1)) break;
                 const int z = (int)(t_begin + 64 * c);
                 const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kb = sbase + (s ? kKB1 : kKB0);
+                GDR2_TRACE_AT(c, 0);
                 mbar_arrive_expect_tx(&bars[B_FULL0 + s], 3 * 16384);
                 for (int blk = 0; blk < 2; ++blk) {
                     void *dst_e = smem + (eq - sbase) + blk * 16384;
@@ -247,19 +319,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         // ---------------- producer: v tiles, L2 prefetch of log_alpha, w -----
         if (lane == 0) {
             int issued = 0;
-            tma_prefetch_3d(&map_la, 0, (int)h, (int)t_begin);
             tma_prefetch_3d(&map_w, 0, (int)h, (int)t_begin);
             for (int c = 0; c < nc; ++c) {
                 if (c >= 1 && !wait_bar(&bars[B_VFREE], (c - 1) & 1, abort_flag, 2)) break;
                 const int z = (int)(t_begin + 64 * c);
+                GDR2_TRACE_AT(c, 1);
                 mbar_arrive_expect_tx(&bars[B_VFULL], 16384);
                 for (int blk = 0; blk < 2; ++blk)
                     tma_load_3d(smem + kZB + blk * 8192, &map_v, &bars[B_VFULL], 64 * blk, (int)h, z);
                 issued = c + 1;
-                if (c + 1 < nc) {
-                    tma_prefetch_3d(&map_la, 0, (int)h, z + 64);
-                    tma_prefetch_3d(&map_w, 0, (int)h, z + 64);
-                }
+                if (c + 1 < nc) tma_prefetch_3d(&map_w, 0, (int)h, z + 64);
             }
             if (issued > 0) {
                 volatile int dummy = 0;
@@ -268,100 +337,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ------------------------------------------
+        // ---------------- MMA issuer for the prep pipeline --------------------
         if (lane == 0) {
             const uint32_t i_ap = idesc_bf16_f32(128, 64, false, false);
             const uint32_t i_w = idesc_bf16_f32(128, 64, true, false);
-            const uint32_t i_us = idesc_bf16_f32(128, 64, false, true, true);
-            const uint32_t i_os = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t i_su = idesc_bf16_f32(128, 128, false, true);
-            int cp = 0, pstep = 0, cc = 0, cstep = 0;
-            uint64_t last_progress = globaltimer_ns();
-            while (cc < nc) {
-                bool progress = false;
-                if (cp < nc) {
-                    const int s = cp & 1;
-                    const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
-                    if (pstep == 0 && mbar_test(&bars[B_PREP], cp & 1)) {
-                        tc_fence_after();
+            for (int cp = 0; cp < nc; ++cp) {
+                const int s = cp & 1;
+                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
+                if (!spin_bar(&bars[B_PREP], cp & 1, abort_flag, 12)) break;
+                tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t a = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                            const uint64_t b = smem_desc_sw128(kbb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                            mma_ss(tb + kTmAPW, a, b, i_ap, kk > 0);
-                        }
-                        tc_commit(&bars[B_AP]);
-                        pstep = 1;
-                        progress = true;
-                    } else if (pstep == 1 && cc > cp - 2 && mbar_test(&bars[B_T], cp & 1)) {
-                        tc_fence_after();
-                        const uint32_t ucol = s ? kTmU1 : kTmU0;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bt = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
-                            const uint64_t ae = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
-                            const uint64_t az = smem_desc_sw128(sbase + kZB + kk * 2048, 8192, 1024);
-                            mma_ss(tb + kTmAPW, ae, bt, i_w, kk > 0);
-                            mma_ss(tb + ucol, az, bt, i_w, kk > 0);
-                        }
-                        tc_commit(&bars[B_WDONE]);
-                        tc_commit(&bars[B_VFREE]);
-                        pstep = 0;
-                        ++cp;
-                        progress = true;
-                    }
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(kbb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tb + kTmAPW, a, b, i_ap, kk > 0);
                 }
-                if (cc < cp) {
-                    const int s = cc & 1;
-                    const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
-                    const uint32_t ucol = s ? kTmU1 : kTmU0;
-                    if (cstep == 0 && mbar_test(&bars[B_WREADY0 + s], (cc >> 1) & 1) &&
-                        mbar_test(&bars[B_SREADY], cc & 1)) {
-                        tc_fence_after();
-                        const uint32_t wb = sbase + (s ? kWB1 : kWB0);
+                tc_commit(&bars[B_AP]);
+                GDR2_TRACE_AT(cp, 2);
+                // U slot (cp % 2) is free once the epilogue has read chunk cp-2's U
+                if (cp >= 2 && !spin_bar(&bars[B_UFREE0 + s], ((cp >> 1) - 1) & 1, abort_flag, 13)) break;
+                if (!spin_bar(&bars[B_T], cp & 1, abort_flag, 14)) break;
+                tc_fence_after();
+                const uint32_t ucol = s ? kTmU1 : kTmU0;
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t bw = smem_desc_sw128(wb + kk * 2048, 8192, 1024);
-                            mma_ts(tb + ucol, tb + kTmSB + kk * 8, bw, i_us, 1);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t bq = smem_desc_sw128(eq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024);
-                            mma_ts(tb + kTmO, tb + kTmSB + kk * 8, bq, i_os, kk > 0);
-                        }
-                        tc_commit(&bars[B_UDONE]);
-                        cstep = 1;
-                        progress = true;
-                    } else if (cstep == 1 && mbar_test(&bars[B_UCONV], cc & 1)) {
-                        tc_fence_after();
-                        const uint32_t pb = sbase + (s ? kPB1 : kPB0);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bp = smem_desc_sw128(pb + kk * 32, 16, 1024);
-                            mma_ts(tb + kTmO, tb + kTmUB + kk * 8, bp, i_os, 1);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bk = smem_desc_sw128(kbb + kk * 2048, 8192, 1024);
-                            mma_ts(tb + kTmMaster, tb + kTmUB + kk * 8, bk, i_su, 1);
-                        }
-                        tc_commit(&bars[B_SDONE]);
-                        tc_commit(&bars[B_SLOTFREE0 + s]);
-                        cstep = 0;
-                        ++cc;
-                        progress = true;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bt = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
+                    const uint64_t ae = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
+                    const uint64_t az = smem_desc_sw128(sbase + kZB + kk * 2048, 8192, 1024);
+                    mma_ss(tb + kTmAPW, ae, bt, i_w, kk > 0);
+                    mma_ss(tb + ucol, az, bt, i_w, kk > 0);
                 }
-                if (progress) {
-                    last_progress = globaltimer_ns();
-                } else {
-                    if (*abort_flag) break;
-                    if (globaltimer_ns() - last_progress > kWaitNs) {
-                        *abort_flag = 1;
-                        atomicCAS(&g_chunk_tc_error, 0, 0x100 | 3);
-                        break;
-                    }
-                }
+                tc_commit(&bars[B_WDONE]);
+                GDR2_TRACE_AT(cp, 3);
+                tc_commit(&bars[B_VFREE]);
             }
             // drain every MMA this thread issued before TMEM is released
             tc_commit(&bars[B_DRAIN]);
@@ -369,109 +377,197 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
             mbar_wait(&bars[B_DRAIN], 0, g2, 22);
         }
+    } else if (warp == 3) {
+        // ---------------- MMA issuer for the state chain -----------------------
+        if (lane == 0) {
+            const uint32_t i_us = idesc_bf16_f32(128, 64, false, true, true);
+            const uint32_t i_os = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t i_su = idesc_bf16_f32(128, 128, false, true);
+            for (int cc = 0; cc < nc; ++cc) {
+                const int s = cc & 1;
+                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
+                const uint32_t ucol = s ? kTmU1 : kTmU0;
+                if (!spin_bar(&bars[B_WREADY0 + s], (cc >> 1) & 1, abort_flag, 15)) break;
+                if (!spin_bar(&bars[B_SREADY], cc & 1, abort_flag, 16)) break;
+                tc_fence_after();
+                const uint32_t wb = sbase + (s ? kWB1 : kWB0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bw = smem_desc_sw128(wb + kk * 2048, 8192, 1024);
+                    mma_ts(tb + ucol, tb + kTmSB + kk * 8, bw, i_us, 1);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bq = smem_desc_sw128(eq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024);
+                    mma_ts(tb + kTmO, tb + kTmSB + kk * 8, bq, i_os, kk > 0);
+                }
+                tc_commit(&bars[B_UDONE]);
+                GDR2_TRACE_AT(cc, 4);
+                if (!spin_bar(&bars[B_UCONV], cc & 1, abort_flag, 17)) break;
+                tc_fence_after();
+                const uint32_t pb = sbase + (s ? kPB1 : kPB0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bp = smem_desc_sw128(pb + kk * 32, 16, 1024);
+                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, bp, i_os, 1);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bk = smem_desc_sw128(kbb + kk * 2048, 8192, 1024);
+                    mma_ts(tb + kTmMaster, tb + kTmUB + kk * 8, bk, i_su, 1);
+                }
+                tc_commit(&bars[B_SDONE]);
+                GDR2_TRACE_AT(cc, 5);
+                tc_commit(&bars[B_SLOTFREE0 + s]);
+            }
+            tc_commit(&bars[B_DRAIN2]);
+            volatile int dummy = 0;
+            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+            mbar_wait(&bars[B_DRAIN2], 0, g2, 23);
+        }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- prep warpgroup ---------------------------------------
+        // Thread layout for the element-wise work: lane g owns key channels
+        // 4g..4g+3 (64-channel block kb = g / 16), warp rb owns rows
+        // 16rb..16rb+15. Loads are unconditional (rows clamped to the valid
+        // range) and rows past the chunk end are zeroed with selects, so the
+        // compiler can keep many loads in flight.
         const int pw = warp - 4, tp = tid - 128;
-        const int kb = pw & 1, hf = pw >> 1;
-        const int p = kb * 32 + lane;          // column pair: channels 2p, 2p+1
-        const int r0 = 32 * hf;
+        const int g = lane, rb = pw, kb = g >> 4;
+        const uint32_t cbyte = 8 * (g & 15);
+        constexpr float kLog2e = 1.4426950408889634f;
+        const float *la_s = reinterpret_cast<const float *>(smem + kSA);  // staged log_alpha [64][128]
+        int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
+        if (tp == 0) {  // log_alpha of chunk 0; later chunks are issued after each inversion
+            ++la_issued;
+            mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
+            tma_load_3d(smem + kSA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)t_begin);
+        }
         for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
+            unsigned char *e_tile = smem + (s ? kEQ1 : kEQ0) + kb * 16384;
+            unsigned char *q_tile = e_tile + 8192;
+            unsigned char *k_tile = smem + (s ? kKB1 : kKB0) + kb * 8192;
 
-            // log-decay of this thread's 32 rows and 2 channels (L2-prefetched)
-            float2 la[32];
+            if (tp == 0) GDR2_TRACE_AT(c, 8);
+            // write-gate rows of this chunk, consumed in the Z step (L2-prefetched)
+            uint2 wv[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = r0 + i;
-                la[i] = r < L ? *reinterpret_cast<const float2 *>(prm.la + ((t0 + r) * H + h) * kD + 2 * p)
-                              : make_float2(0.f, 0.f);
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * rb + i;
+                const int rr = r < L ? r : L - 1;
+                wv[i] = *reinterpret_cast<const uint2 *>(prm.w + ((t0 + rr) * H + h) * kD + 4 * g);
             }
-            // d_r = g_r - g_31: suffix sums (first half), prefix sums (second half)
-            float2 tot = make_float2(0.f, 0.f);
-            if (hf == 0) {
+            // log-decay of 16 rows x 4 channels from the TMA-staged tile, masked past L
+            if (!group_and(kBarPrep, wait_bar(&bars[B_LAFULL], c & 1, abort_flag, 18))) break;
+            float4 la[16];
 #pragma unroll
-                for (int i = 31; i >= 0; --i) {
-                    const float2 x = la[i];
-                    la[i] = make_float2(-tot.x, -tot.y);
-                    tot.x += x.x;
-                    tot.y += x.y;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    tot.x += la[i].x;
-                    tot.y += la[i].y;
-                    la[i] = tot;
-                }
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * rb + i;
+                const float4 x = *reinterpret_cast<const float4 *>(la_s + r * 128 + 4 * g);
+                la[i] = r < L ? x : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            float *vt = (hf == 0 ? vecT0 : vecT1) + (c & 3) * 128;
-            vt[2 * p] = tot.x;
-            vt[2 * p + 1] = tot.y;
+            float4 bs = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                bs.x += la[i].x; bs.y += la[i].y; bs.z += la[i].z; bs.w += la[i].w;
+            }
+            *reinterpret_cast<float4 *>(vecBS + rb * 128 + 4 * g) = bs;
+            if (tp == 0) GDR2_TRACE_AT(c, 25);
 
+            if (tp == 0) GDR2_TRACE_AT(c, 9);
+            // (this group barrier also publishes the block sums)
             if (!group_and(kBarPrep, wait_bar(&bars[B_FULL0 + s], (c >> 1) & 1, abort_flag, 4))) break;
-            // factors, in place: b -> Em, q -> Qm, k -> Km
+            if (tp == 0) GDR2_TRACE_AT(c, 10);
+            // d_r = g_r - g_31 in log2 units: suffix sums for rows < 32, prefix
+            // sums for rows >= 32; half sums T0 = g_31, T1 = g_63 - g_31.
             {
-                const uint32_t e_tile = eq + kb * 16384, q_tile = e_tile + 8192;
-                const uint32_t k_tile = kbb + kb * 8192;
-                const uint32_t byte = 4 * lane;  // channel pair within the 64-wide block
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = r0 + i;
-                    const uint32_t off = sw128_offset(r, byte);
-                    uint32_t oq = 0, ok = 0, oe = 0;
-                    if (r < L) {
-                        const float2 qv = bf2_to_f2(ld_shared_u32(q_tile + off));
-                        const float2 kv = bf2_to_f2(ld_shared_u32(k_tile + off));
-                        const float2 bv = bf2_to_f2(ld_shared_u32(e_tile + off));
-                        const float ux = __expf(la[i].x), uy = __expf(la[i].y);
-                        const float dx = __expf(-la[i].x), dy = __expf(-la[i].y);
-                        oq = pack_bf16x2(qv.x * ux, qv.y * uy);
-                        ok = pack_bf16x2(kv.x * dx, kv.y * dy);
-                        oe = pack_bf16x2(bv.x * kv.x * ux, bv.y * kv.y * uy);
-                    }
-                    st_shared_u32(q_tile + off, oq);
-                    st_shared_u32(k_tile + off, ok);
-                    st_shared_u32(e_tile + off, oe);
+                float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rb == 0) run = *reinterpret_cast<const float4 *>(vecBS + 1 * 128 + 4 * g);
+                if (rb == 3) run = *reinterpret_cast<const float4 *>(vecBS + 2 * 128 + 4 * g);
+                if (rb == 1 || rb == 2) {
+                    const float4 o4 = *reinterpret_cast<const float4 *>(vecBS + (rb == 1 ? 0 : 3) * 128 + 4 * g);
+                    float *vt = (rb == 1 ? vecT0 : vecT1) + (c & 3) * 128 + 4 * g;
+                    *reinterpret_cast<float4 *>(vt) =
+                        make_float4(bs.x + o4.x, bs.y + o4.y, bs.z + o4.z, bs.w + o4.w);
                 }
+                if (rb < 2) {
+#pragma unroll
+                    for (int i = 15; i >= 0; --i) {
+                        const float4 x = la[i];
+                        la[i] = make_float4(-run.x * kLog2e, -run.y * kLog2e, -run.z * kLog2e, -run.w * kLog2e);
+                        run.x += x.x; run.y += x.y; run.z += x.z; run.w += x.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        run.x += la[i].x; run.y += la[i].y; run.z += la[i].z; run.w += la[i].w;
+                        la[i] = make_float4(run.x * kLog2e, run.y * kLog2e, run.z * kLog2e, run.w * kLog2e);
+                    }
+                }
+            }
+            // factors, in place: b -> Em, q -> Qm, k -> Km
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * rb + i;
+                const uint32_t off = sw128_offset(r, cbyte);
+                const uint2 qr = *reinterpret_cast<const uint2 *>(q_tile + off);
+                const uint2 kr = *reinterpret_cast<const uint2 *>(k_tile + off);
+                const uint2 br = *reinterpret_cast<const uint2 *>(e_tile + off);
+                const float2 q0 = bf2_to_f2(qr.x), q1 = bf2_to_f2(qr.y);
+                const float2 k0 = bf2_to_f2(kr.x), k1 = bf2_to_f2(kr.y);
+                const float2 b0 = bf2_to_f2(br.x), b1 = bf2_to_f2(br.y);
+                const float u0 = ex2_approx(la[i].x), u1 = ex2_approx(la[i].y);
+                const float u2 = ex2_approx(la[i].z), u3 = ex2_approx(la[i].w);
+                const float v0 = ex2_approx(-la[i].x), v1 = ex2_approx(-la[i].y);
+                const float v2 = ex2_approx(-la[i].z), v3 = ex2_approx(-la[i].w);
+                const bool ok = r < L;
+                uint2 oq, okk, oe;
+                oq.x = ok ? pack_bf16x2(q0.x * u0, q0.y * u1) : 0u;
+                oq.y = ok ? pack_bf16x2(q1.x * u2, q1.y * u3) : 0u;
+                okk.x = ok ? pack_bf16x2(k0.x * v0, k0.y * v1) : 0u;
+                okk.y = ok ? pack_bf16x2(k1.x * v2, k1.y * v3) : 0u;
+                oe.x = ok ? pack_bf16x2(b0.x * k0.x * u0, b0.y * k0.y * u1) : 0u;
+                oe.y = ok ? pack_bf16x2(b1.x * k1.x * u2, b1.y * k1.y * u3) : 0u;
+                *reinterpret_cast<uint2 *>(q_tile + off) = oq;
+                *reinterpret_cast<uint2 *>(k_tile + off) = okk;
+                *reinterpret_cast<uint2 *>(e_tile + off) = oe;
+                if (i == 7 && tp == 0) GDR2_TRACE_AT(c, 26);
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, 128);
             if (tp == 0) {
+                GDR2_TRACE_AT(c, 11);
                 mbar_arrive(&bars[B_PREP]);
                 mbar_arrive(&bars[B_VEC0 + s]);
             }
 
-            // Z = w . v in place (v tile from TMA, w from global / L2)
+            // Z = w . v in place (v tile from TMA, w loaded at the chunk start)
             {
-                uint32_t wv[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = r0 + i;
-                    wv[i] = r < L ? *reinterpret_cast<const uint32_t *>(prm.w + ((t0 + r) * H + h) * kD + 2 * p)
-                                  : 0u;
-                }
                 if (!group_and(kBarPrep, wait_bar(&bars[B_VFULL], c & 1, abort_flag, 5))) break;
-                const uint32_t z_tile = sbase + kZB + kb * 8192;
+                unsigned char *z_tile = smem + kZB + kb * 8192;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = r0 + i;
-                    const uint32_t off = sw128_offset(r, 4 * lane);
-                    uint32_t oz = 0;
-                    if (r < L) {
-                        const float2 vv = bf2_to_f2(ld_shared_u32(z_tile + off));
-                        const float2 ww = bf2_to_f2(wv[i]);
-                        oz = pack_bf16x2(vv.x * ww.x, vv.y * ww.y);
-                    }
-                    st_shared_u32(z_tile + off, oz);
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * rb + i;
+                    const uint32_t off = sw128_offset(r, cbyte);
+                    const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
+                    const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
+                    const float2 w0 = bf2_to_f2(wv[i].x), w1 = bf2_to_f2(wv[i].y);
+                    const bool ok = r < L;
+                    uint2 oz;
+                    oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
+                    oz.y = ok ? pack_bf16x2(v1.x * w1.x, v1.y * w1.y) : 0u;
+                    *reinterpret_cast<uint2 *>(z_tile + off) = oz;
                 }
             }
             fence_proxy_async_smem();
 
             // [A; P] from TMEM: lanes 0-63 rows of A, lanes 64-127 rows of P
+            if (tp == 0) GDR2_TRACE_AT(c, 12);
             if (!group_and(kBarPrep, wait_bar(&bars[B_AP], c & 1, abort_flag, 6))) break;
+            if (tp == 0) GDR2_TRACE_AT(c, 13);
             tc_fence_after();
             {
                 const uint32_t taddr = tb + kTmAPW + ((uint32_t)(32 * pw) << 16);
@@ -479,13 +575,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
                 tc_wait_ld();
-                if (pw < 2) {
+                if (pw < 2) {  // A^T[s][r] = A[r][s] for s < r
                     const int r = 32 * pw + lane;
-                    float *row = sA + r * 65;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        row[j] = j < r ? __uint_as_float(v0[j]) : 0.f;
-                        row[32 + j] = 32 + j < r ? __uint_as_float(v1[j]) : 0.f;
+                        sA[j * kLD + r] = j < r ? __uint_as_float(v0[j]) : 0.f;
+                        sA[(32 + j) * kLD + r] = 32 + j < r ? __uint_as_float(v1[j]) : 0.f;
                     }
                 } else {
                     const int r = 32 * (pw - 2) + lane;
@@ -495,80 +590,123 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         x[j] = j <= r ? __uint_as_float(v0[j]) : 0.f;
                         x[32 + j] = 32 + j <= r ? __uint_as_float(v1[j]) : 0.f;
                     }
-                    store_row_bf16_sw128(sbase + (s ? kPB1 : kPB0), r, x);
+                    store_row_bf16_sw128(smem + (s ? kPB1 : kPB0), r, x);
                 }
             }
             named_bar_sync(kBarPrep, 128);
 
-            // T = (I + A)^{-1}: two 32x32 diagonal blocks by column-wise forward
-            // substitution, then T10 = -T11 (A10 T00).
+            if (tp == 0) GDR2_TRACE_AT(c, 14);
+            // T = (I + A)^{-1} by doubling on 16-row blocks (A held transposed,
+            // sA = A^T; T in sT, both fp32 with row pitch kLD):
+            //   1. T_ii = (I + A_ii)^{-1} for the four 16x16 diagonal blocks,
+            //      right-looking forward substitution, one column per thread;
+            //   2. inside each 32-block: T_10 = -T_11 (A_10 T_00);
+            //   3. across the two 32-blocks: T_10 = -T_11 (A_10 T_00).
+            // Products of step 2 and 3 park their intermediate Y in the
+            // upper-right (zero) part of T, which the bf16 writer masks out.
             if (tp < 64) {
-                const int j = tp, base = (j >> 5) * 32, jj = j & 31;
-                float x[32];
+                const int blk = tp >> 4, jj = tp & 15, base = 16 * blk;
+                float x[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float *arow = sA + (base + i) * 65 + base;
-                    float acc = (i == jj) ? 1.f : 0.f;
+                for (int i = 0; i < 16; ++i) x[i] = (i == jj) ? 1.f : 0.f;
 #pragma unroll
-                    for (int s2 = 0; s2 < i; ++s2) acc = fmaf(-arow[s2], x[s2], acc);
-                    x[i] = acc;
+                for (int i = 0; i < 15; ++i) {
+                    const float xi = x[i];
+                    const float *at = sA + (base + i) * kLD + base;
+                    float a16[16];
+#pragma unroll
+                    for (int q4 = (i + 1) >> 2; q4 < 4; ++q4) {
+                        const float4 v = *reinterpret_cast<const float4 *>(at + 4 * q4);
+                        a16[4 * q4] = v.x; a16[4 * q4 + 1] = v.y; a16[4 * q4 + 2] = v.z; a16[4 * q4 + 3] = v.w;
+                    }
+#pragma unroll
+                    for (int k2 = i + 1; k2 < 16; ++k2) x[k2] = fmaf(-a16[k2], xi, x[k2]);
                 }
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sT[(base + i) * 65 + j] = x[i];
-            }
-            named_bar_sync(kBarPrep, 128);
-            {   // Y = A10 T00 -> scratch in the (unused) upper-right block of sT
-                const int i = tp >> 2, j0 = (tp & 3) * 8;
-                float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                const float *arow = sA + (32 + i) * 65;
-#pragma unroll 4
-                for (int kx = 0; kx < 32; ++kx) {
-                    const float a = arow[kx];
-                    const float *trow = sT + kx * 65 + j0;
+                for (int i = 0; i < 16; ++i) sT[(base + i) * kLD + base + jj] = x[i];
+                if ((blk & 1) == 0) {  // the upper-right 16x16 of each 32-block is zero
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) y[q] = fmaf(a, trow[q], y[q]);
+                    for (int i = 0; i < 16; ++i) sT[(base + i) * kLD + base + 16 + jj] = 0.f;
                 }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) sT[i * 65 + 32 + j0 + q] = y[q];
             }
             named_bar_sync(kBarPrep, 128);
-            {   // T10 = -T11 Y
-                const int i = tp >> 2, j0 = (tp & 3) * 8;
-                float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                const float *trow = sT + (32 + i) * 65 + 32;
-#pragma unroll 4
-                for (int kx = 0; kx < 32; ++kx) {
-                    const float t = trow[kx];
-                    const float *yrow = sT + kx * 65 + 32 + j0;
+            if (tp == 0) GDR2_TRACE_AT(c, 27);
+            // Steps 2 and 3 are small dense products: warp-level tensor-core
+            // MMAs in tf32 with fp32 accumulation (T itself is consumed in
+            // bf16 afterwards, so tf32 products lose nothing that matters).
+            {   // step 2a: Y = A_10 T_00 inside 32-block pb (warp: pb = pw >> 1, n-tile pw & 1)
+                const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                // A_10(i, k) = A[b0+16+i][b0+k] = sA[(b0+k) * kLD + b0+16+i]
+                tile_tf32<16>(d, sA + b0 * kLD + b0 + 16, 1, kLD, sT + b0 * kLD + b0 + 8 * nt, kLD, lane);
+                store_tile(d, sT + (16 * pb) * kLD + 32 + 16 * pb + 8 * nt, kLD, lane, 1.f);
+            }
+            named_bar_sync(kBarPrep, 128);
+            {   // step 2b: T_10 = -T_11 Y inside 32-block pb
+                const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_tf32<16>(d, sT + (b0 + 16) * kLD + b0 + 16, kLD, 1,
+                              sT + (16 * pb) * kLD + 32 + 16 * pb + 8 * nt, kLD, lane);
+                store_tile(d, sT + (b0 + 16) * kLD + b0 + 8 * nt, kLD, lane, -1.f);
+            }
+            named_bar_sync(kBarPrep, 128);
+            {   // step 3a: Y = A_10 T_00 across the 32-blocks -> upper-right 32x32 of sT
+                const int mt = pw >> 1;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) y[q] = fmaf(-t, yrow[q], y[q]);
+                for (int q = 0; q < 2; ++q) {
+                    const int nt = 2 * (pw & 1) + q;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    // A_10(i, k) = A[32+i][k] = sA[k * kLD + 32+i]
+                    tile_tf32<32>(d, sA + 32 + 16 * mt, 1, kLD, sT + 8 * nt, kLD, lane);
+                    store_tile(d, sT + (16 * mt) * kLD + 32 + 8 * nt, kLD, lane, 1.f);
                 }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) sT[(32 + i) * 65 + j0 + q] = y[q];
             }
             named_bar_sync(kBarPrep, 128);
+            if (tp == 0) GDR2_TRACE_AT(c, 28);
+            {   // step 3b: T_10 = -T_11 Y
+                const int mt = pw >> 1;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int nt = 2 * (pw & 1) + q;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_tf32<32>(d, sT + (32 + 16 * mt) * kLD + 32, kLD, 1, sT + 32 + 8 * nt, kLD, lane);
+                    store_tile(d, sT + (32 + 16 * mt) * kLD + 8 * nt, kLD, lane, -1.f);
+                }
+            }
+            named_bar_sync(kBarPrep, 128);
+            if (tp == 0) GDR2_TRACE_AT(c, 29);
             {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
                 const int r = tp >> 1, half = tp & 1;
-                const float *trow = sT + r * 65 + 32 * half;
+                const float *trow = sT + r * kLD + 32 * half;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    uint32_t u[4];
+                    uint32_t ue[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int s0 = 32 * half + 8 * q + 2 * e;
-                        u[e] = pack_bf16x2(s0 <= r ? trow[8 * q + 2 * e] : 0.f,
-                                           s0 + 1 <= r ? trow[8 * q + 2 * e + 1] : 0.f);
+                        ue[e] = pack_bf16x2(s0 <= r ? trow[8 * q + 2 * e] : 0.f,
+                                            s0 + 1 <= r ? trow[8 * q + 2 * e + 1] : 0.f);
                     }
-                    st_shared_v4(sbase + kTB + sw128_offset(r, 64 * half + 16 * q), u[0], u[1], u[2], u[3]);
+                    *reinterpret_cast<uint4 *>(smem + kTB + sw128_offset(r, 64 * half + 16 * q)) =
+                        make_uint4(ue[0], ue[1], ue[2], ue[3]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarPrep, 128);
-            if (tp == 0) mbar_arrive(&bars[B_T]);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 15);
+                mbar_arrive(&bars[B_T]);
+                if (c + 1 < nc) {  // the inversion scratch is free again: stage the next log_alpha
+                    ++la_issued;
+                    mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
+                    tma_load_3d(smem + kSA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)(t0 + 64));
+                }
+            }
 
             // W^T (lanes = key channels) -> bf16 smem operand, MN-major rows
             if (!group_and(kBarPrep, wait_bar(&bars[B_WDONE], c & 1, abort_flag, 7))) break;
+            if (tp == 0) GDR2_TRACE_AT(c, 16);
             tc_fence_after();
             {
                 const uint32_t taddr = tb + kTmAPW + ((uint32_t)(32 * pw) << 16);
@@ -582,12 +720,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     x[j] = __uint_as_float(v0[j]);
                     x[32 + j] = __uint_as_float(v1[j]);
                 }
-                store_row_bf16_sw128(sbase + (s ? kWB1 : kWB0), 32 * pw + lane, x);
+                store_row_bf16_sw128(smem + (s ? kWB1 : kWB0), 32 * pw + lane, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarPrep, 128);
-            if (tp == 0) mbar_arrive(&bars[B_WREADY0 + s]);
+            if (tp == 0) { GDR2_TRACE_AT(c, 17); mbar_arrive(&bars[B_WREADY0 + s]); }
+        }
+        if (tp == 0 && la_issued > 0) {  // drain a staged log_alpha load still in flight
+            volatile int dummy = 0;
+            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+            mbar_wait(&bars[B_LAFULL], (la_issued - 1) & 1, g2, 24);
         }
     } else if (warp >= 8) {
         // ---------------- epilogue warpgroup -----------------------------------
@@ -626,6 +769,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
             // U^T (fp32) -> bf16 pairs in TMEM for the second MMA group
             if (!group_and(kBarEpi, wait_bar(&bars[B_UDONE], c & 1, abort_flag, 9))) break;
+            if (te == 0) GDR2_TRACE_AT(c, 20);
             tc_fence_after();
             {
                 uint32_t v0[32], v1[32], ub[16];
@@ -645,24 +789,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             tc_fence_before();
             named_bar_sync(kBarEpi, 128);
-            if (te == 0) mbar_arrive(&bars[B_UCONV]);
+            if (te == 0) {
+                GDR2_TRACE_AT(c, 21);
+                mbar_arrive(&bars[B_UCONV]);
+                mbar_arrive(&bars[B_UFREE0 + s]);
+            }
 
             if (!group_and(kBarEpi, wait_bar(&bars[B_SDONE], c & 1, abort_flag, 10))) break;
+            if (te == 0) GDR2_TRACE_AT(c, 22);
             tc_fence_after();
-            {   // o rows of this chunk
+            // O^T row j -> registers as bf16 pairs (rows r, r+1); stored after the
+            // state hand-off so the global stores stay off the chunk-to-chunk path
+            uint32_t opk[32];
+            {
                 uint32_t v0[32], v1[32];
                 tmem_ld32(tb + kTmO + lane_off, v0);
                 tmem_ld32(tb + kTmO + lane_off + 32, v1);
                 tc_wait_ld();
-                __nv_bfloat16 *orow = prm.o + (t0 * H + h) * kD + j;
-                const int64_t rstride = H * kD;
 #pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    if (r < L) orow[r * rstride] = __float2bfloat16_rn(__uint_as_float(v0[r]));
-#pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    if (32 + r < L) orow[(32 + r) * rstride] = __float2bfloat16_rn(__uint_as_float(v1[r]));
+                for (int q = 0; q < 16; ++q) {
+                    opk[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
+                    opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
+                }
             }
+            if (te == 0) GDR2_TRACE_AT(c, 23);
             // state scale: e^{g_C - g_31} and, unless last, e^{g'_31} of the next chunk
             const bool last = (c + 1 == nc);
             // (the group barrier also means everyone is done reading vecF)
@@ -672,30 +822,58 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             vecF[j] = expf(vecT1[(c & 3) * 128 + j] + (last ? 0.f : vecT0[((c + 1) & 3) * 128 + j]));
             named_bar_sync(kBarEpi, 128);
 #pragma unroll 1
-            for (int g4 = 0; g4 < 4; ++g4) {
-                uint32_t m[32];
-                tmem_ld32(tb + kTmMaster + lane_off + 32 * g4, m);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t m0[32], m1[32];
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
                 tc_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    m[q] = __float_as_uint(__uint_as_float(m[q]) * vecF[32 * g4 + q]);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 f0 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 4 * q);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 32 + 4 * q);
+                    m0[4 * q + 0] = __float_as_uint(__uint_as_float(m0[4 * q + 0]) * f0.x);
+                    m0[4 * q + 1] = __float_as_uint(__uint_as_float(m0[4 * q + 1]) * f0.y);
+                    m0[4 * q + 2] = __float_as_uint(__uint_as_float(m0[4 * q + 2]) * f0.z);
+                    m0[4 * q + 3] = __float_as_uint(__uint_as_float(m0[4 * q + 3]) * f0.w);
+                    m1[4 * q + 0] = __float_as_uint(__uint_as_float(m1[4 * q + 0]) * f1.x);
+                    m1[4 * q + 1] = __float_as_uint(__uint_as_float(m1[4 * q + 1]) * f1.y);
+                    m1[4 * q + 2] = __float_as_uint(__uint_as_float(m1[4 * q + 2]) * f1.z);
+                    m1[4 * q + 3] = __float_as_uint(__uint_as_float(m1[4 * q + 3]) * f1.w);
+                }
                 if (!last) {
-                    uint32_t sbf[16];
+                    uint32_t s0b[16], s1b[16];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        sbf[q] = pack_bf16x2(__uint_as_float(m[2 * q]), __uint_as_float(m[2 * q + 1]));
-                    tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
-                    tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
+                    for (int q = 0; q < 16; ++q) {
+                        s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
+                        s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
+                    }
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
                 } else if (prm.final_state) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        prm.final_state[state_base + (int64_t)(32 * g4 + q) * kD + j] = __uint_as_float(m[q]);
+                    for (int q = 0; q < 32; ++q) {
+                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
+                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
+                    }
                 }
             }
             tc_wait_st();
             tc_fence_before();
             named_bar_sync(kBarEpi, 128);
+            if (te == 0) GDR2_TRACE_AT(c, 24);
             if (!last && te == 0) mbar_arrive(&bars[B_SREADY]);
+            {   // o rows of this chunk
+                __nv_bfloat16 *orow = prm.o + (t0 * H + h) * kD + j;
+                const int64_t rstride = H * kD;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162 *>(&opk[q]);
+                    if (2 * q < L) orow[(2 * q) * rstride] = pr.x;
+                    if (2 * q + 1 < L) orow[(2 * q + 1) * rstride] = pr.y;
+                }
+            }
         }
     }
 

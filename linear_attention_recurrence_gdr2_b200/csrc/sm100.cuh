@@ -56,13 +56,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
+// Potentially blocking probe: the thread may be suspended (up to ~100 us)
+// until the phase completes, so waiting warps take no issue slots.
 __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(100000u) : "memory");
     return ok != 0;
 }
 
@@ -81,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     uint32_t spins = 0;
     while (!mbar_try(bar, parity)) {
         if (*g.abort_flag) return false;
-        if ((++spins & 63u) == 0 && globaltimer_ns() > g.deadline_ns) {
+        if ((++spins & 7u) == 0 && globaltimer_ns() > g.deadline_ns) {
             *g.abort_flag = 1;
             atomicCAS(g.error_word, 0, 0x100 | site);
             return false;

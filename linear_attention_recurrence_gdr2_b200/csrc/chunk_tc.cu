@@ -18,27 +18,33 @@
 //
 // One CTA owns one (sequence, head) and walks its chunks in order. Everything
 // is computed transposed so that the value dimension (128) sits on the MMA's
-// M axis and on the 128 TMEM lanes:
-//     [A; P]    = [Em; Qm] Km^T                      (M=128, N=64,  K=128)
-//     W^T       = Em^T T^T,   U0^T = Z^T T^T         (M=128, N=64,  K=64)
-//     U^T       = U0^T - Sm^T W^T,  O^T = Sm^T Qm^T  (A = Sm^T from TMEM)
-//     O^T      += U^T P^T,  M^T += U^T Km            (A = U^T from TMEM)
+// M axis and on the 128 TMEM lanes (P = tril(Qm Km^T), M = the TMEM state):
+//     [A; P]        = [Em; Qm] Km^T                 M=128 N=64  K=128
+//     W^T, U0^T     = Em^T T^T, Z^T T^T             M=128 N=64  K=64 (x2)
+//     [U^T | O^T]  += Sm^T [-W; Qm]^T               M=128 N=128 K=128, A in TMEM
+//     [O^T | M^T]  += U^T [P^T | Km]                M=128 N=192 K=64,  A in TMEM
+// Merging the products that share an A operand into one wide-N chain keeps
+// the number of tcgen05.mma instructions per chunk at 28 (each costs a fixed
+// issue time whatever its N). -W is written K-major over Em (dead by then) so
+// that it sits right before Qm; P^T is written MN-major right before Km; the
+// O columns sit between U and the state in TMEM.
 // The fp32 state lives in TMEM (as M = Diag(e^{g_31}) S plus the chunk's
 // update); once per chunk the epilogue scales it by e^{g_C - g_31 + g'_31}
 // (g'_31: the next chunk's half sum) and writes its bf16 copy back to TMEM as
 // the next chunk's MMA operand.
 //
-// Warp roles (12 warps):
+// Warp roles (16 warps; the first warpgroup gives registers to the others):
 //   0      TMA producer of q, k, b tiles (double-buffered slots)
 //   1      tcgen05.mma issuer of the prep pipeline ([A;P], W^T, U0^T)
-//   2      TMEM allocator; TMA producer of v tiles and L2 prefetch of
-//          log_alpha and w
-//   3      tcgen05.mma issuer of the state chain (U^T, O^T, state update)
-//   4..7   prep: cumulative decay, factors, Z, (I + A)^{-1}, W^T to smem
-//   8..11  epilogue: U^T to bf16, o stores, state scaling, final state
-// Every wait is bounded: after about a second without progress the CTA
-// records the site in the device error word and winds down (drains its TMA
-// loads and MMAs, frees TMEM, returns).
+//   2      TMEM allocator; TMA producer of v tiles, L2 prefetch of w
+//   3      tcgen05.mma issuer of the state chain
+//   4..7   prep A: cumulative decay, decay-absorbed factors, Z, P^T
+//   8..11  prep B: (I + A)^{-1}, -W
+//   12..15 epilogue: U^T to bf16, o stores, state scaling, final state
+// The two prep warpgroups work on consecutive chunks concurrently, and both
+// run ahead of the state chain. Every wait is bounded: after about a second
+// without progress the CTA records the site in the device error word and
+// winds down (drains its TMA loads and MMAs, frees TMEM, returns).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -68,48 +74,47 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreadsTC = 384;
+constexpr int kThreadsTC = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;  // one second per wait
 
 // ---- shared memory map (bytes from the 1024-aligned base) ----------------
-constexpr uint32_t kEQ0 = 0;             // [kb0: Em 8K | Qm 8K][kb1: Em 8K | Qm 8K]
+constexpr uint32_t kEQ0 = 0;             // per 64-channel block kb: [Em -> -W 8K | Qm 8K]
 constexpr uint32_t kEQ1 = 32768;
-constexpr uint32_t kKB0 = 65536;         // Km: [kb0 8K][kb1 8K]
-constexpr uint32_t kKB1 = 81920;
-constexpr uint32_t kZB = 98304;          // v -> Z: [dv block 0 8K][dv block 1 8K]
-constexpr uint32_t kTB = 114688;         // T bf16, 64 rows x 128 B
-constexpr uint32_t kPB0 = 122880;        // P bf16, 64 rows x 128 B
-constexpr uint32_t kPB1 = 131072;
-constexpr uint32_t kWB0 = 139264;        // W^T bf16, 128 rows x 128 B
-constexpr uint32_t kWB1 = 155648;
+constexpr uint32_t kKB0 = 65536;         // [P 8K | Km kb0 8K | Km kb1 8K]
+constexpr uint32_t kKB1 = 90112;
+constexpr uint32_t kKmOff = 8192;        // Km after the P block
+constexpr uint32_t kZB0 = 114688;        // v -> Z: [dv block 0 8K][dv block 1 8K]
+constexpr uint32_t kZB1 = 131072;
+constexpr uint32_t kTB = 147456;         // T bf16, 64 rows x 128 B
+constexpr uint32_t kLA = 155648;         // staged log_alpha, fp32 [64][128]
 constexpr int kLD = 68;                  // fp32 scratch row pitch (16-byte aligned rows)
-constexpr uint32_t kSA = 172032;         // fp32 A^T, 64 x kLD
+constexpr uint32_t kSA = 188416;         // fp32 A^T, 64 x kLD
 constexpr uint32_t kST = kSA + 64 * kLD * 4;  // fp32 T, 64 x kLD
 constexpr uint32_t kVEC = kST + 64 * kLD * 4; // half sums: T0[4][128], T1[4][128], f[128]
 constexpr uint32_t kBSUM = kVEC + (8 * 128 + 128) * 4;  // per-row-block log-decay sums [4][128]
 constexpr uint32_t kBAR = kBSUM + 4 * 128 * 4;
-constexpr int kNumBars = 23;
+constexpr int kNumBars = 28;
 constexpr uint32_t kMISC = kBAR + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kMISC + 64 + 1024;  // + alignment slack
 
 // barrier indices
 enum {
-    B_FULL0 = 0, B_FULL1, B_SLOTFREE0, B_SLOTFREE1, B_VFULL, B_VFREE, B_PREP, B_AP, B_T,
-    B_WDONE, B_WREADY0, B_WREADY1, B_SREADY, B_UDONE, B_UCONV, B_SDONE, B_VEC0, B_VEC1,
-    B_DRAIN, B_DRAIN2, B_UFREE0, B_UFREE1, B_LAFULL
+    B_FULL0 = 0, B_FULL1, B_SLOTFREE0, B_SLOTFREE1, B_VFULL0, B_VFULL1, B_VFREE0, B_VFREE1,
+    B_LAFULL, B_PREP, B_VEC0, B_VEC1, B_AP, B_AFREE, B_ZREADY0, B_ZREADY1, B_T, B_WDONE, B_WREADY0,
+    B_WREADY1, B_PREADY0, B_PREADY1, B_SREADY, B_UDONE, B_UCONV, B_SDONE, B_DRAIN, B_DRAIN2
 };
 
-// ---- TMEM column map ------------------------------------------------------
-constexpr uint32_t kTmMaster = 0;    // fp32 state (transposed), 128 columns
-constexpr uint32_t kTmO = 128;       // O^T fp32, 64
-constexpr uint32_t kTmU0 = 192;      // U^T fp32 slots, 64 each
-constexpr uint32_t kTmU1 = 256;
-constexpr uint32_t kTmAPW = 320;     // [A;P] then W^T, fp32, 64
+// ---- TMEM column map (512 columns allocated) -------------------------------
+constexpr uint32_t kTmU = 0;         // U^T fp32, 64      } one N=128 accumulator
+constexpr uint32_t kTmO = 64;        // O^T fp32, 64      }        } one N=192
+constexpr uint32_t kTmMaster = 128;  // state (transposed) fp32, 128 } accumulator
+constexpr uint32_t kTmAP = 256;      // [A; P] fp32, 64
+constexpr uint32_t kTmW = 320;       // W^T fp32, 64
 constexpr uint32_t kTmSB = 384;      // Sm^T bf16 pairs, 64 words
 constexpr uint32_t kTmUB = 448;      // U^T bf16 pairs, 32 words
 
-// prep / epilogue named barriers
-constexpr uint32_t kBarPrep = 1, kBarEpi = 2;
+// group (named) barriers
+constexpr uint32_t kBarPrepA = 1, kBarEpi = 2, kBarPrepB = 3;
 
 struct TcParams {
     const float *la;
@@ -222,6 +227,9 @@ __device__ __forceinline__ void store_row_bf16_sw128(unsigned char *tile, uint32
     }
 }
 
+__device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory"); }
+__device__ __forceinline__ void setmaxnreg_inc152() { asm volatile("setmaxnreg.inc.sync.aligned.u32 152;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreadsTC, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_v,
@@ -285,6 +293,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     const uint32_t tb = *tmem_slot;
 
     // =====================================================================
+    if (warp < 4) {
+    setmaxnreg_dec40();
     if (warp == 0) {
         // ---------------- producer: q, k, b tiles ----------------------------
         if (lane == 0) {
@@ -293,48 +303,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const int s = c & 1;
                 if (c >= 2 && !wait_bar(&bars[B_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, 1)) break;
                 const int z = (int)(t_begin + 64 * c);
-                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kb = sbase + (s ? kKB1 : kKB0);
+                unsigned char *eq = smem + (s ? kEQ1 : kEQ0), *kq = smem + (s ? kKB1 : kKB0) + kKmOff;
                 GDR2_TRACE_AT(c, 0);
                 mbar_arrive_expect_tx(&bars[B_FULL0 + s], 3 * 16384);
                 for (int blk = 0; blk < 2; ++blk) {
-                    void *dst_e = smem + (eq - sbase) + blk * 16384;
-                    void *dst_q = smem + (eq - sbase) + blk * 16384 + 8192;
-                    void *dst_k = smem + (kb - sbase) + blk * 8192;
-                    tma_load_3d(dst_e, &map_b, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
-                    tma_load_3d(dst_q, &map_q, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
-                    tma_load_3d(dst_k, &map_k, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
+                    tma_load_3d(eq + blk * 16384, &map_b, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
+                    tma_load_3d(eq + blk * 16384 + 8192, &map_q, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
+                    tma_load_3d(kq + blk * 8192, &map_k, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
                 }
                 issued[s] = (c >> 1) + 1;
             }
             // drain: wait (bounded) for every load issued into each slot
             for (int s = 0; s < 2; ++s)
                 if (issued[s] > 0) {
-                    WaitGuard g{globaltimer_ns() + kWaitNs, abort_flag, &g_chunk_tc_error};
                     volatile int dummy = 0;
-                    WaitGuard g2{g.deadline_ns, &dummy, &g_chunk_tc_error};
+                    WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
                     mbar_wait(&bars[B_FULL0 + s], (issued[s] - 1) & 1, g2, 20);
                 }
         }
     } else if (warp == 2) {
-        // ---------------- producer: v tiles, L2 prefetch of log_alpha, w -----
+        // ---------------- producer: v tiles, L2 prefetch of w ------------------
         if (lane == 0) {
-            int issued = 0;
             tma_prefetch_3d(&map_w, 0, (int)h, (int)t_begin);
+            int vissued[2] = {0, 0};
             for (int c = 0; c < nc; ++c) {
-                if (c >= 1 && !wait_bar(&bars[B_VFREE], (c - 1) & 1, abort_flag, 2)) break;
+                const int s = c & 1;
+                if (c >= 2 && !wait_bar(&bars[B_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, 2)) break;
                 const int z = (int)(t_begin + 64 * c);
                 GDR2_TRACE_AT(c, 1);
-                mbar_arrive_expect_tx(&bars[B_VFULL], 16384);
+                mbar_arrive_expect_tx(&bars[B_VFULL0 + s], 16384);
                 for (int blk = 0; blk < 2; ++blk)
-                    tma_load_3d(smem + kZB + blk * 8192, &map_v, &bars[B_VFULL], 64 * blk, (int)h, z);
-                issued = c + 1;
+                    tma_load_3d(smem + (s ? kZB1 : kZB0) + blk * 8192, &map_v, &bars[B_VFULL0 + s], 64 * blk,
+                                (int)h, z);
+                vissued[s] = (c >> 1) + 1;
                 if (c + 1 < nc) tma_prefetch_3d(&map_w, 0, (int)h, z + 64);
             }
-            if (issued > 0) {
-                volatile int dummy = 0;
-                WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-                mbar_wait(&bars[B_VFULL], (issued - 1) & 1, g2, 21);
-            }
+            for (int s = 0; s < 2; ++s)
+                if (vissued[s] > 0) {
+                    volatile int dummy = 0;
+                    WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+                    mbar_wait(&bars[B_VFULL0 + s], (vissued[s] - 1) & 1, g2, 21);
+                }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer for the prep pipeline --------------------
@@ -343,33 +352,37 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const uint32_t i_w = idesc_bf16_f32(128, 64, true, false);
             for (int cp = 0; cp < nc; ++cp) {
                 const int s = cp & 1;
-                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
-                if (!spin_bar(&bars[B_PREP], cp & 1, abort_flag, 12)) break;
+                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
+                const uint32_t km = sbase + (s ? kKB1 : kKB0) + kKmOff;
+                if (!wait_bar(&bars[B_PREP], cp & 1, abort_flag, 12)) break;
+                if (cp >= 1 && !wait_bar(&bars[B_AFREE], (cp - 1) & 1, abort_flag, 13)) break;
                 tc_fence_after();
+                // [A; P] = [Em; Qm] Km^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t a = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(kbb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tb + kTmAPW, a, b, i_ap, kk > 0);
+                    const uint64_t b = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tb + kTmAP, a, b, i_ap, kk > 0);
                 }
                 tc_commit(&bars[B_AP]);
                 GDR2_TRACE_AT(cp, 2);
-                // U slot (cp % 2) is free once the epilogue has read chunk cp-2's U
-                if (cp >= 2 && !spin_bar(&bars[B_UFREE0 + s], ((cp >> 1) - 1) & 1, abort_flag, 13)) break;
-                if (!spin_bar(&bars[B_T], cp & 1, abort_flag, 14)) break;
+                if (!wait_bar(&bars[B_T], cp & 1, abort_flag, 14)) break;
+                if (!wait_bar(&bars[B_ZREADY0 + s], (cp >> 1) & 1, abort_flag, 15)) break;
+                // the single U region is free once the epilogue has read chunk cp-1's U
+                if (cp >= 1 && !wait_bar(&bars[B_UCONV], (cp - 1) & 1, abort_flag, 16)) break;
                 tc_fence_after();
-                const uint32_t ucol = s ? kTmU1 : kTmU0;
+                // W^T = Em^T T^T, U0^T = Z^T T^T
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bt = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
                     const uint64_t ae = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
-                    const uint64_t az = smem_desc_sw128(sbase + kZB + kk * 2048, 8192, 1024);
-                    mma_ss(tb + kTmAPW, ae, bt, i_w, kk > 0);
-                    mma_ss(tb + ucol, az, bt, i_w, kk > 0);
+                    const uint64_t az = smem_desc_sw128(sbase + (s ? kZB1 : kZB0) + kk * 2048, 8192, 1024);
+                    mma_ss(tb + kTmW, ae, bt, i_w, kk > 0);
+                    mma_ss(tb + kTmU, az, bt, i_w, kk > 0);
                 }
                 tc_commit(&bars[B_WDONE]);
                 GDR2_TRACE_AT(cp, 3);
-                tc_commit(&bars[B_VFREE]);
+                tc_commit(&bars[B_VFREE0 + s]);
             }
             // drain every MMA this thread issued before TMEM is released
             tc_commit(&bars[B_DRAIN]);
@@ -380,41 +393,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     } else if (warp == 3) {
         // ---------------- MMA issuer for the state chain -----------------------
         if (lane == 0) {
-            const uint32_t i_us = idesc_bf16_f32(128, 64, false, true, true);
-            const uint32_t i_os = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t i_su = idesc_bf16_f32(128, 128, false, true);
+            const uint32_t i_uo = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t i_op = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t i_mk = idesc_bf16_f32(128, 128, false, true);
             for (int cc = 0; cc < nc; ++cc) {
                 const int s = cc & 1;
-                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0), kbb = sbase + (s ? kKB1 : kKB0);
-                const uint32_t ucol = s ? kTmU1 : kTmU0;
-                if (!spin_bar(&bars[B_WREADY0 + s], (cc >> 1) & 1, abort_flag, 15)) break;
-                if (!spin_bar(&bars[B_SREADY], cc & 1, abort_flag, 16)) break;
+                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
+                const uint32_t kbs = sbase + (s ? kKB1 : kKB0);
+                if (!wait_bar(&bars[B_WREADY0 + s], (cc >> 1) & 1, abort_flag, 17)) break;
+                if (!wait_bar(&bars[B_SREADY], cc & 1, abort_flag, 18)) break;
+                GDR2_TRACE_AT(cc, 7);
                 tc_fence_after();
-                const uint32_t wb = sbase + (s ? kWB1 : kWB0);
+                // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bw = smem_desc_sw128(wb + kk * 2048, 8192, 1024);
-                    mma_ts(tb + ucol, tb + kTmSB + kk * 8, bw, i_us, 1);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bq = smem_desc_sw128(eq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024);
-                    mma_ts(tb + kTmO, tb + kTmSB + kk * 8, bq, i_os, kk > 0);
+                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, b, i_uo, 1);
                 }
                 tc_commit(&bars[B_UDONE]);
                 GDR2_TRACE_AT(cc, 4);
-                if (!spin_bar(&bars[B_UCONV], cc & 1, abort_flag, 17)) break;
+                if (!wait_bar(&bars[B_UCONV], cc & 1, abort_flag, 19)) break;
+                if (!wait_bar(&bars[B_PREADY0 + s], (cc >> 1) & 1, abort_flag, 25)) break;
+                GDR2_TRACE_AT(cc, 6);
                 tc_fence_after();
-                const uint32_t pb = sbase + (s ? kPB1 : kPB0);
+                // O^T += U^T P^T (B = P, K-major), M^T += U^T Km (B = Km, MN-major)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bp = smem_desc_sw128(pb + kk * 32, 16, 1024);
-                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, bp, i_os, 1);
+                    const uint64_t b = smem_desc_sw128(kbs + kk * 32, 16, 1024);
+                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, b, i_op, 1);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bk = smem_desc_sw128(kbb + kk * 2048, 8192, 1024);
-                    mma_ts(tb + kTmMaster, tb + kTmUB + kk * 8, bk, i_su, 1);
+                    const uint64_t b = smem_desc_sw128(kbs + kKmOff + kk * 2048, 8192, 1024);
+                    mma_ts(tb + kTmMaster, tb + kTmUB + kk * 8, b, i_mk, 1);
                 }
                 tc_commit(&bars[B_SDONE]);
                 GDR2_TRACE_AT(cc, 5);
@@ -425,23 +436,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
             mbar_wait(&bars[B_DRAIN2], 0, g2, 23);
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ---------------- prep warpgroup ---------------------------------------
-        // Thread layout for the element-wise work: lane g owns key channels
-        // 4g..4g+3 (64-channel block kb = g / 16), warp rb owns rows
-        // 16rb..16rb+15. Loads are unconditional (rows clamped to the valid
-        // range) and rows past the chunk end are zeroed with selects, so the
-        // compiler can keep many loads in flight.
+    }
+    } else if (warp < 8) {
+        setmaxnreg_inc152();
+        // ---------------- prep A: decay factors, Z, P^T ------------------------
+        // Element-wise layout: lane g owns key channels 4g..4g+3 (64-channel
+        // block kb = g / 16), warp rb owns rows 16rb..16rb+15. Loads are
+        // unconditional (rows clamped to the valid range) and rows past the
+        // chunk end are zeroed with selects, so many loads stay in flight.
         const int pw = warp - 4, tp = tid - 128;
         const int g = lane, rb = pw, kb = g >> 4;
         const uint32_t cbyte = 8 * (g & 15);
         constexpr float kLog2e = 1.4426950408889634f;
-        const float *la_s = reinterpret_cast<const float *>(smem + kSA);  // staged log_alpha [64][128]
+        const float *la_s = reinterpret_cast<const float *>(smem + kLA);  // staged log_alpha [64][128]
         int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
-        if (tp == 0) {  // log_alpha of chunk 0; later chunks are issued after each inversion
+        if (tp == 0) {
             ++la_issued;
             mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
-            tma_load_3d(smem + kSA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)t_begin);
+            tma_load_3d(smem + kLA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)t_begin);
         }
         for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
@@ -449,7 +461,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
             unsigned char *e_tile = smem + (s ? kEQ1 : kEQ0) + kb * 16384;
             unsigned char *q_tile = e_tile + 8192;
-            unsigned char *k_tile = smem + (s ? kKB1 : kKB0) + kb * 8192;
+            unsigned char *k_tile = smem + (s ? kKB1 : kKB0) + kKmOff + kb * 8192;
 
             if (tp == 0) GDR2_TRACE_AT(c, 8);
             // write-gate rows of this chunk, consumed in the Z step (L2-prefetched)
@@ -460,8 +472,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const int rr = r < L ? r : L - 1;
                 wv[i] = *reinterpret_cast<const uint2 *>(prm.w + ((t0 + rr) * H + h) * kD + 4 * g);
             }
-            // log-decay of 16 rows x 4 channels from the TMA-staged tile, masked past L
-            if (!group_and(kBarPrep, wait_bar(&bars[B_LAFULL], c & 1, abort_flag, 18))) break;
+            if (!group_and(kBarPrepA, wait_bar(&bars[B_LAFULL], c & 1, abort_flag, 3))) break;
             float4 la[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -475,12 +486,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 bs.x += la[i].x; bs.y += la[i].y; bs.z += la[i].z; bs.w += la[i].w;
             }
             *reinterpret_cast<float4 *>(vecBS + rb * 128 + 4 * g) = bs;
-            if (tp == 0) GDR2_TRACE_AT(c, 25);
-
             if (tp == 0) GDR2_TRACE_AT(c, 9);
-            // (this group barrier also publishes the block sums)
-            if (!group_and(kBarPrep, wait_bar(&bars[B_FULL0 + s], (c >> 1) & 1, abort_flag, 4))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 10);
+            // (this group barrier also publishes the block sums and frees the staging tile)
+            fence_proxy_async_smem();
+            if (!group_and(kBarPrepA, wait_bar(&bars[B_FULL0 + s], (c >> 1) & 1, abort_flag, 4))) break;
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 10);
+                if (c + 1 < nc) {  // stage the next chunk's log_alpha
+                    ++la_issued;
+                    mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
+                    tma_load_3d(smem + kLA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)(t0 + 64));
+                }
+            }
             // d_r = g_r - g_31 in log2 units: suffix sums for rows < 32, prefix
             // sums for rows >= 32; half sums T0 = g_31, T1 = g_63 - g_31.
             {
@@ -534,10 +551,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 *reinterpret_cast<uint2 *>(q_tile + off) = oq;
                 *reinterpret_cast<uint2 *>(k_tile + off) = okk;
                 *reinterpret_cast<uint2 *>(e_tile + off) = oe;
-                if (i == 7 && tp == 0) GDR2_TRACE_AT(c, 26);
             }
             fence_proxy_async_smem();
-            named_bar_sync(kBarPrep, 128);
+            named_bar_sync(kBarPrepA, 128);
             if (tp == 0) {
                 GDR2_TRACE_AT(c, 11);
                 mbar_arrive(&bars[B_PREP]);
@@ -546,8 +562,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
             // Z = w . v in place (v tile from TMA, w loaded at the chunk start)
             {
-                if (!group_and(kBarPrep, wait_bar(&bars[B_VFULL], c & 1, abort_flag, 5))) break;
-                unsigned char *z_tile = smem + kZB + kb * 8192;
+                if (!group_and(kBarPrepA, wait_bar(&bars[B_VFULL0 + s], (c >> 1) & 1, abort_flag, 5))) break;
+                unsigned char *z_tile = smem + (s ? kZB1 : kZB0) + kb * 8192;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * rb + i;
@@ -563,47 +579,80 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             fence_proxy_async_smem();
+            named_bar_sync(kBarPrepA, 128);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 12);
+                mbar_arrive(&bars[B_ZREADY0 + s]);
+            }
 
-            // [A; P] from TMEM: lanes 0-63 rows of A, lanes 64-127 rows of P
-            if (tp == 0) GDR2_TRACE_AT(c, 12);
-            if (!group_and(kBarPrep, wait_bar(&bars[B_AP], c & 1, abort_flag, 6))) break;
+            // P = tril(Qm Km^T) from TMEM lanes 64-127 -> K-major rows before Km
+            if (!group_and(kBarPrepA, wait_bar(&bars[B_AP], c & 1, abort_flag, 6))) break;
             if (tp == 0) GDR2_TRACE_AT(c, 13);
             tc_fence_after();
-            {
-                const uint32_t taddr = tb + kTmAPW + ((uint32_t)(32 * pw) << 16);
+            if (pw >= 2) {
+                const uint32_t taddr = tb + kTmAP + ((uint32_t)(32 * pw) << 16);
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
                 tc_wait_ld();
-                if (pw < 2) {  // A^T[s][r] = A[r][s] for s < r
-                    const int r = 32 * pw + lane;
+                const int r = 32 * (pw - 2) + lane;
+                float x[64];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        sA[j * kLD + r] = j < r ? __uint_as_float(v0[j]) : 0.f;
-                        sA[(32 + j) * kLD + r] = 32 + j < r ? __uint_as_float(v1[j]) : 0.f;
-                    }
-                } else {
-                    const int r = 32 * (pw - 2) + lane;
-                    float x[64];
+                for (int j2 = 0; j2 < 32; ++j2) {
+                    x[j2] = j2 <= r ? __uint_as_float(v0[j2]) : 0.f;
+                    x[32 + j2] = 32 + j2 <= r ? __uint_as_float(v1[j2]) : 0.f;
+                }
+                store_row_bf16_sw128(smem + (s ? kKB1 : kKB0), r, x);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarPrepA, 128);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 14);
+                mbar_arrive(&bars[B_PREADY0 + s]);
+            }
+        }
+        if (tp == 0 && la_issued > 0) {  // drain a staged log_alpha load still in flight
+            volatile int dummy = 0;
+            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+            mbar_wait(&bars[B_LAFULL], (la_issued - 1) & 1, g2, 24);
+        }
+    } else if (warp < 12) {
+        setmaxnreg_inc152();
+        // ---------------- prep B: (I + A)^{-1}, -W ------------------------------
+        const int pw = warp - 8, tp = tid - 256;
+        for (int c = 0; c < nc; ++c) {
+            const int s = c & 1;
+            if (!group_and(kBarPrepB, wait_bar(&bars[B_AP], c & 1, abort_flag, 7))) break;
+            if (tp == 0) GDR2_TRACE_AT(c, 15);
+            tc_fence_after();
+            if (pw < 2) {  // A rows (TMEM lanes 0-63) -> A^T[s][r] for s < r
+                const uint32_t taddr = tb + kTmAP + ((uint32_t)(32 * pw) << 16);
+                uint32_t v0[32], v1[32];
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tc_wait_ld();
+                const int r = 32 * pw + lane;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        x[j] = j <= r ? __uint_as_float(v0[j]) : 0.f;
-                        x[32 + j] = 32 + j <= r ? __uint_as_float(v1[j]) : 0.f;
-                    }
-                    store_row_bf16_sw128(smem + (s ? kPB1 : kPB0), r, x);
+                for (int j = 0; j < 32; ++j) {
+                    sA[j * kLD + r] = j < r ? __uint_as_float(v0[j]) : 0.f;
+                    sA[(32 + j) * kLD + r] = 32 + j < r ? __uint_as_float(v1[j]) : 0.f;
                 }
             }
-            named_bar_sync(kBarPrep, 128);
+            tc_fence_before();
+            named_bar_sync(kBarPrepB, 128);
+            if (tp == 0) mbar_arrive(&bars[B_AFREE]);
 
-            if (tp == 0) GDR2_TRACE_AT(c, 14);
             // T = (I + A)^{-1} by doubling on 16-row blocks (A held transposed,
             // sA = A^T; T in sT, both fp32 with row pitch kLD):
             //   1. T_ii = (I + A_ii)^{-1} for the four 16x16 diagonal blocks,
             //      right-looking forward substitution, one column per thread;
             //   2. inside each 32-block: T_10 = -T_11 (A_10 T_00);
             //   3. across the two 32-blocks: T_10 = -T_11 (A_10 T_00).
-            // Products of step 2 and 3 park their intermediate Y in the
-            // upper-right (zero) part of T, which the bf16 writer masks out.
+            // Steps 2 and 3 are small dense products run as warp-level tensor-core
+            // MMAs in tf32 with fp32 accumulation (T itself is consumed in bf16),
+            // their intermediate Y parked in the upper-right (zero) part of T,
+            // which the bf16 writer masks out.
             if (tp < 64) {
                 const int blk = tp >> 4, jj = tp & 15, base = 16 * blk;
                 float x[16];
@@ -629,19 +678,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     for (int i = 0; i < 16; ++i) sT[(base + i) * kLD + base + 16 + jj] = 0.f;
                 }
             }
-            named_bar_sync(kBarPrep, 128);
-            if (tp == 0) GDR2_TRACE_AT(c, 27);
-            // Steps 2 and 3 are small dense products: warp-level tensor-core
-            // MMAs in tf32 with fp32 accumulation (T itself is consumed in
-            // bf16 afterwards, so tf32 products lose nothing that matters).
+            named_bar_sync(kBarPrepB, 128);
             {   // step 2a: Y = A_10 T_00 inside 32-block pb (warp: pb = pw >> 1, n-tile pw & 1)
                 const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                // A_10(i, k) = A[b0+16+i][b0+k] = sA[(b0+k) * kLD + b0+16+i]
                 tile_tf32<16>(d, sA + b0 * kLD + b0 + 16, 1, kLD, sT + b0 * kLD + b0 + 8 * nt, kLD, lane);
                 store_tile(d, sT + (16 * pb) * kLD + 32 + 16 * pb + 8 * nt, kLD, lane, 1.f);
             }
-            named_bar_sync(kBarPrep, 128);
+            named_bar_sync(kBarPrepB, 128);
             {   // step 2b: T_10 = -T_11 Y inside 32-block pb
                 const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -649,20 +693,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                               sT + (16 * pb) * kLD + 32 + 16 * pb + 8 * nt, kLD, lane);
                 store_tile(d, sT + (b0 + 16) * kLD + b0 + 8 * nt, kLD, lane, -1.f);
             }
-            named_bar_sync(kBarPrep, 128);
+            named_bar_sync(kBarPrepB, 128);
             {   // step 3a: Y = A_10 T_00 across the 32-blocks -> upper-right 32x32 of sT
                 const int mt = pw >> 1;
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int nt = 2 * (pw & 1) + q;
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    // A_10(i, k) = A[32+i][k] = sA[k * kLD + 32+i]
                     tile_tf32<32>(d, sA + 32 + 16 * mt, 1, kLD, sT + 8 * nt, kLD, lane);
                     store_tile(d, sT + (16 * mt) * kLD + 32 + 8 * nt, kLD, lane, 1.f);
                 }
             }
-            named_bar_sync(kBarPrep, 128);
-            if (tp == 0) GDR2_TRACE_AT(c, 28);
+            named_bar_sync(kBarPrepB, 128);
             {   // step 3b: T_10 = -T_11 Y
                 const int mt = pw >> 1;
 #pragma unroll
@@ -673,8 +715,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     store_tile(d, sT + (32 + 16 * mt) * kLD + 8 * nt, kLD, lane, -1.f);
                 }
             }
-            named_bar_sync(kBarPrep, 128);
-            if (tp == 0) GDR2_TRACE_AT(c, 29);
+            named_bar_sync(kBarPrepB, 128);
             {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
                 const int r = tp >> 1, half = tp & 1;
                 const float *trow = sT + r * kLD + 32 * half;
@@ -692,54 +733,52 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(kBarPrep, 128);
+            named_bar_sync(kBarPrepB, 128);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 15);
+                GDR2_TRACE_AT(c, 16);
                 mbar_arrive(&bars[B_T]);
-                if (c + 1 < nc) {  // the inversion scratch is free again: stage the next log_alpha
-                    ++la_issued;
-                    mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
-                    tma_load_3d(smem + kSA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)(t0 + 64));
-                }
             }
 
-            // W^T (lanes = key channels) -> bf16 smem operand, MN-major rows
-            if (!group_and(kBarPrep, wait_bar(&bars[B_WDONE], c & 1, abort_flag, 7))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 16);
+            // W^T (lanes = key channels) -> -W, K-major, into the Em half of the slot
+            if (!group_and(kBarPrepB, wait_bar(&bars[B_WDONE], c & 1, abort_flag, 8))) break;
+            if (tp == 0) GDR2_TRACE_AT(c, 17);
             tc_fence_after();
             {
-                const uint32_t taddr = tb + kTmAPW + ((uint32_t)(32 * pw) << 16);
+                const uint32_t taddr = tb + kTmW + ((uint32_t)(32 * pw) << 16);
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
                 tc_wait_ld();
-                float x[64];
+                const int ch = 32 * pw + lane;
+                unsigned char *wt = smem + (s ? kEQ1 : kEQ0) + (ch >> 6) * 16384;
+                const uint32_t cb = 2 * (ch & 63);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    x[j] = __uint_as_float(v0[j]);
-                    x[32 + j] = __uint_as_float(v1[j]);
+                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(j, cb)) =
+                        __float2bfloat16_rn(-__uint_as_float(v0[j]));
+                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 + j, cb)) =
+                        __float2bfloat16_rn(-__uint_as_float(v1[j]));
                 }
-                store_row_bf16_sw128(smem + (s ? kWB1 : kWB0), 32 * pw + lane, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar_sync(kBarPrep, 128);
-            if (tp == 0) { GDR2_TRACE_AT(c, 17); mbar_arrive(&bars[B_WREADY0 + s]); }
+            named_bar_sync(kBarPrepB, 128);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 18);
+                mbar_arrive(&bars[B_WREADY0 + s]);
+            }
         }
-        if (tp == 0 && la_issued > 0) {  // drain a staged log_alpha load still in flight
-            volatile int dummy = 0;
-            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-            mbar_wait(&bars[B_LAFULL], (la_issued - 1) & 1, g2, 24);
-        }
-    } else if (warp >= 8) {
+    } else {
+        setmaxnreg_inc152();
         // ---------------- epilogue warpgroup -----------------------------------
-        const int ew = warp - 8, te = tid - 256;
+        const int ew = warp - 12, te = tid - 384;
         const int j = 32 * ew + lane;                       // value channel = TMEM lane
         const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
+        const uint32_t zeros[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                    0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         bool ok = true;
-        // master = Diag(e^{g_31 of chunk 0}) S0  (transposed: row j over key channels)
-        ok = group_and(kBarEpi, wait_bar(&bars[B_VEC0], 0, abort_flag, 8));
+        // master = Diag(e^{g_31 of chunk 0}) S0  (transposed: row j over key channels); O = 0
+        ok = group_and(kBarEpi, wait_bar(&bars[B_VEC0], 0, abort_flag, 9));
         if (ok) {
             vecF[j] = expf(vecT0[j]);
             named_bar_sync(kBarEpi, 128);
@@ -758,24 +797,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
                 tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
             }
+            tmem_st32(tb + kTmO + lane_off, zeros);
+            tmem_st32(tb + kTmO + lane_off + 32, zeros);
             tc_wait_st();
             tc_fence_before();
             named_bar_sync(kBarEpi, 128);
             if (te == 0) mbar_arrive(&bars[B_SREADY]);
         }
         for (int c = 0; ok && c < nc; ++c) {
-            const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            // U^T (fp32) -> bf16 pairs in TMEM for the second MMA group
-            if (!group_and(kBarEpi, wait_bar(&bars[B_UDONE], c & 1, abort_flag, 9))) break;
+            // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
+            if (!group_and(kBarEpi, wait_bar(&bars[B_UDONE], c & 1, abort_flag, 10))) break;
             if (te == 0) GDR2_TRACE_AT(c, 20);
             tc_fence_after();
             {
                 uint32_t v0[32], v1[32], ub[16];
-                const uint32_t ucol = s ? kTmU1 : kTmU0;
-                tmem_ld32(tb + ucol + lane_off, v0);
-                tmem_ld32(tb + ucol + lane_off + 32, v1);
+                tmem_ld32(tb + kTmU + lane_off, v0);
+                tmem_ld32(tb + kTmU + lane_off + 32, v1);
                 tc_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 16; ++q)
@@ -792,14 +831,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (te == 0) {
                 GDR2_TRACE_AT(c, 21);
                 mbar_arrive(&bars[B_UCONV]);
-                mbar_arrive(&bars[B_UFREE0 + s]);
             }
 
-            if (!group_and(kBarEpi, wait_bar(&bars[B_SDONE], c & 1, abort_flag, 10))) break;
+            if (!group_and(kBarEpi, wait_bar(&bars[B_SDONE], c & 1, abort_flag, 11))) break;
             if (te == 0) GDR2_TRACE_AT(c, 22);
             tc_fence_after();
-            // O^T row j -> registers as bf16 pairs (rows r, r+1); stored after the
-            // state hand-off so the global stores stay off the chunk-to-chunk path
+            // O^T row j -> registers as bf16 pairs (rows r, r+1), then the O region
+            // is zeroed for the next chunk; o is stored after the state hand-off
             uint32_t opk[32];
             {
                 uint32_t v0[32], v1[32];
@@ -812,51 +850,43 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
                 }
             }
+            const bool last = (c + 1 == nc);
+            if (!last) {
+                tmem_st32(tb + kTmO + lane_off, zeros);
+                tmem_st32(tb + kTmO + lane_off + 32, zeros);
+            }
             if (te == 0) GDR2_TRACE_AT(c, 23);
             // state scale: e^{g_C - g_31} and, unless last, e^{g'_31} of the next chunk
-            const bool last = (c + 1 == nc);
             // (the group barrier also means everyone is done reading vecF)
             if (!group_and(kBarEpi, last || wait_bar(&bars[B_VEC0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1,
-                                                      abort_flag, 11)))
+                                                      abort_flag, 26)))
                 break;
             vecF[j] = expf(vecT1[(c & 3) * 128 + j] + (last ? 0.f : vecT0[((c + 1) & 3) * 128 + j]));
             named_bar_sync(kBarEpi, 128);
 #pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t m0[32], m1[32];
-                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+            for (int g4 = 0; g4 < 4; ++g4) {
+                uint32_t m[32];
+                tmem_ld32(tb + kTmMaster + lane_off + 32 * g4, m);
                 tc_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 f0 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 4 * q);
-                    const float4 f1 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 32 + 4 * q);
-                    m0[4 * q + 0] = __float_as_uint(__uint_as_float(m0[4 * q + 0]) * f0.x);
-                    m0[4 * q + 1] = __float_as_uint(__uint_as_float(m0[4 * q + 1]) * f0.y);
-                    m0[4 * q + 2] = __float_as_uint(__uint_as_float(m0[4 * q + 2]) * f0.z);
-                    m0[4 * q + 3] = __float_as_uint(__uint_as_float(m0[4 * q + 3]) * f0.w);
-                    m1[4 * q + 0] = __float_as_uint(__uint_as_float(m1[4 * q + 0]) * f1.x);
-                    m1[4 * q + 1] = __float_as_uint(__uint_as_float(m1[4 * q + 1]) * f1.y);
-                    m1[4 * q + 2] = __float_as_uint(__uint_as_float(m1[4 * q + 2]) * f1.z);
-                    m1[4 * q + 3] = __float_as_uint(__uint_as_float(m1[4 * q + 3]) * f1.w);
+                    const float4 f = *reinterpret_cast<const float4 *>(vecF + 32 * g4 + 4 * q);
+                    m[4 * q + 0] = __float_as_uint(__uint_as_float(m[4 * q + 0]) * f.x);
+                    m[4 * q + 1] = __float_as_uint(__uint_as_float(m[4 * q + 1]) * f.y);
+                    m[4 * q + 2] = __float_as_uint(__uint_as_float(m[4 * q + 2]) * f.z);
+                    m[4 * q + 3] = __float_as_uint(__uint_as_float(m[4 * q + 3]) * f.w);
                 }
                 if (!last) {
-                    uint32_t s0b[16], s1b[16];
+                    uint32_t sbf[16];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
-                        s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
-                    }
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
-                    tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
-                    tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
+                    for (int q = 0; q < 16; ++q)
+                        sbf[q] = pack_bf16x2(__uint_as_float(m[2 * q]), __uint_as_float(m[2 * q + 1]));
+                    tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
+                    tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
                 } else if (prm.final_state) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
-                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
-                    }
+                    for (int q = 0; q < 32; ++q)
+                        prm.final_state[state_base + (int64_t)(32 * g4 + q) * kD + j] = __uint_as_float(m[q]);
                 }
             }
             tc_wait_st();

@@ -641,7 +641,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             tc_fence_before();
             named_bar_sync(kBarPrepB, 128);
-            if (tp == 0) mbar_arrive(&bars[B_AFREE]);
+            if (tp == 0) { GDR2_TRACE_AT(c, 25); mbar_arrive(&bars[B_AFREE]); }
 
             // T = (I + A)^{-1} by doubling on 16-row blocks (A held transposed,
             // sA = A^T; T in sT, both fp32 with row pitch kLD):
@@ -679,6 +679,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             named_bar_sync(kBarPrepB, 128);
+            if (tp == 0) GDR2_TRACE_AT(c, 26);
             {   // step 2a: Y = A_10 T_00 inside 32-block pb (warp: pb = pw >> 1, n-tile pw & 1)
                 const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -716,6 +717,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             named_bar_sync(kBarPrepB, 128);
+            if (tp == 0) GDR2_TRACE_AT(c, 27);
             {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
                 const int r = tp >> 1, half = tp & 1;
                 const float *trow = sT + r * kLD + 32 * half;
@@ -864,29 +866,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             vecF[j] = expf(vecT1[(c & 3) * 128 + j] + (last ? 0.f : vecT0[((c + 1) & 3) * 128 + j]));
             named_bar_sync(kBarEpi, 128);
 #pragma unroll 1
-            for (int g4 = 0; g4 < 4; ++g4) {
-                uint32_t m[32];
-                tmem_ld32(tb + kTmMaster + lane_off + 32 * g4, m);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t m0[32], m1[32];
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
                 tc_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 f = *reinterpret_cast<const float4 *>(vecF + 32 * g4 + 4 * q);
-                    m[4 * q + 0] = __float_as_uint(__uint_as_float(m[4 * q + 0]) * f.x);
-                    m[4 * q + 1] = __float_as_uint(__uint_as_float(m[4 * q + 1]) * f.y);
-                    m[4 * q + 2] = __float_as_uint(__uint_as_float(m[4 * q + 2]) * f.z);
-                    m[4 * q + 3] = __float_as_uint(__uint_as_float(m[4 * q + 3]) * f.w);
+                    const float4 f0 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 4 * q);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 32 + 4 * q);
+                    m0[4 * q + 0] = __float_as_uint(__uint_as_float(m0[4 * q + 0]) * f0.x);
+                    m0[4 * q + 1] = __float_as_uint(__uint_as_float(m0[4 * q + 1]) * f0.y);
+                    m0[4 * q + 2] = __float_as_uint(__uint_as_float(m0[4 * q + 2]) * f0.z);
+                    m0[4 * q + 3] = __float_as_uint(__uint_as_float(m0[4 * q + 3]) * f0.w);
+                    m1[4 * q + 0] = __float_as_uint(__uint_as_float(m1[4 * q + 0]) * f1.x);
+                    m1[4 * q + 1] = __float_as_uint(__uint_as_float(m1[4 * q + 1]) * f1.y);
+                    m1[4 * q + 2] = __float_as_uint(__uint_as_float(m1[4 * q + 2]) * f1.z);
+                    m1[4 * q + 3] = __float_as_uint(__uint_as_float(m1[4 * q + 3]) * f1.w);
                 }
                 if (!last) {
-                    uint32_t sbf[16];
+                    uint32_t s0b[16], s1b[16];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        sbf[q] = pack_bf16x2(__uint_as_float(m[2 * q]), __uint_as_float(m[2 * q + 1]));
-                    tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
-                    tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
+                    for (int q = 0; q < 16; ++q) {
+                        s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
+                        s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
+                    }
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
                 } else if (prm.final_state) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        prm.final_state[state_base + (int64_t)(32 * g4 + q) * kD + j] = __uint_as_float(m[q]);
+                    for (int q = 0; q < 32; ++q) {
+                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
+                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
+                    }
                 }
             }
             tc_wait_st();
@@ -894,14 +908,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             named_bar_sync(kBarEpi, 128);
             if (te == 0) GDR2_TRACE_AT(c, 24);
             if (!last && te == 0) mbar_arrive(&bars[B_SREADY]);
-            {   // o rows of this chunk
-                __nv_bfloat16 *orow = prm.o + (t0 * H + h) * kD + j;
+            {   // o rows of this chunk: adjacent lanes (channels j, j+1) trade halves so
+                // that the even lane stores rows 2q and the odd lane rows 2q+1 as
+                // 4-byte (j, j+1) pairs
+                const bool odd = (lane & 1) != 0;
+                __nv_bfloat16 *obase = prm.o + (t0 * H + h) * kD + (j & ~1);
                 const int64_t rstride = H * kD;
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162 *>(&opk[q]);
-                    if (2 * q < L) orow[(2 * q) * rstride] = pr.x;
-                    if (2 * q + 1 < L) orow[(2 * q + 1) * rstride] = pr.y;
+                    const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel j
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
+                    const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+                    const int r = 2 * q + (odd ? 1 : 0);
+                    if (r < L) *reinterpret_cast<uint32_t *>(obase + r * rstride) = pr;
                 }
             }
         }

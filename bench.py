@@ -133,6 +133,24 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def reduce_max(x: float, device=None) -> float:
+    """Max of a per-rank number over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own replica of the
+    workload, so the job moves world x tokens_per_rank tokens in the slowest
+    rank's time."""
+    return world * tokens_per_rank / (max_ms * 1e-3)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -236,12 +254,7 @@ def main():
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dev)
 
     hbm_peak, _, peak_src = load_peaks()
     inp, label = workload(args.workload)
@@ -328,12 +341,12 @@ def main():
             e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
             h2d = sum(x.numel() * x.element_size() for x in pinned.values())
             d2h = o.numel() * o.element_size() + sf.numel() * sf.element_size()
-            e2e = {"value": world * inp.num_tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+            e2e = {"value": aggregate_throughput(inp.num_tokens, world, e2e_ms), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "ms_per_step": e2e_ms}
 
     ms_per_step = total_ms / args.steps
-    value = world * inp.num_tokens / (ms_per_step * 1e-3)
+    value = aggregate_throughput(inp.num_tokens, world, ms_per_step)
     kern_ms = statistics.mean(per)
     nbytes = chunk_bytes(inp)
     achieved = nbytes / (kern_ms * 1e-3) / 1e9

@@ -113,7 +113,11 @@ int gdr2_version(void);
  *                before it writes its final state)
  *   workspace, workspace_bytes
  *                device scratch of at least gdr2_chunk_fwd_workspace_size()
- *                bytes (NULL allowed when that size is 0)
+ *                bytes, 16-byte aligned (NULL allowed when that size is 0).
+ *                A packed batch of several sequences uses it for the order in
+ *                which sequences are processed (longest first, computed on the
+ *                device from cu_seqlens); its contents are overwritten, so
+ *                calls that share a workspace must be ordered on the GPU.
  *   stream       cudaStream_t
  * Precision: with GDR2_FP32 every product runs in fp32 on CUDA cores; with
  * GDR2_BF16 the dense intra-chunk contractions run on the tensor cores with
@@ -127,7 +131,9 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v,
                            void *o, float *final_state, void *workspace,
                            size_t workspace_bytes, void *stream);
 
-/* Scratch bytes gdr2_chunk_fwd needs for this problem (written to *bytes). */
+/* Scratch bytes gdr2_chunk_fwd needs for this problem (written to *bytes):
+ * 0 for fixed-length batches; a small multiple of 256 bytes (4 bytes per
+ * sequence) for a packed batch of num_seqs > 1 sequences (B == 1). */
 gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
                                           int64_t d_k, int64_t d_v,
                                           int64_t num_seqs, gdr2_dtype dtype,

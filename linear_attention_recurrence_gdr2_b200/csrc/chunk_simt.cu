@@ -58,7 +58,7 @@ chunk_simt_kernel(ChunkArgs args)
     const int tid = threadIdx.x;
     const int j0 = blockIdx.x * kDVT;      // first value column of this tile
     const int64_t h = blockIdx.y;
-    const int64_t n = blockIdx.z;
+    const int64_t n = args.order ? (int64_t)args.order[blockIdx.z] : (int64_t)blockIdx.z;
     const int64_t H = args.H;
     const int DV = (int)args.dv;
 

@@ -121,6 +121,7 @@ struct TcParams {
     const __nv_bfloat16 *w;
     const float *init_state;
     const int32_t *cu_seqlens;
+    const int32_t *order;
     __nv_bfloat16 *o;
     float *final_state;
     int64_t T, H;
@@ -253,7 +254,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = prm.H;
-    const int64_t n = blockIdx.x / H, h = blockIdx.x % H;
+    const int64_t h = blockIdx.x % H;
+    const int64_t n = prm.order ? (int64_t)prm.order[blockIdx.x / H] : (int64_t)(blockIdx.x / H);
     int64_t t_begin, t_end;
     if (prm.cu_seqlens) {
         t_begin = prm.cu_seqlens[n];
@@ -994,6 +996,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.w = (const __nv_bfloat16 *)a.w;
     p.init_state = a.init_state;
     p.cu_seqlens = a.cu_seqlens;
+    p.order = a.order;
     p.o = (__nv_bfloat16 *)a.o;
     p.final_state = a.final_state;
     p.T = a.T;

@@ -48,7 +48,9 @@ gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H, int64
     if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
     gdr2_status st = check_dims(d_k, d_v);
     if (st != GDR2_OK) return st;
-    *bytes = 0;
+    // A packed batch of several sequences (the only case with num_seqs != B)
+    // needs room for its longest-first processing order.
+    *bytes = (B == 1 && num_seqs > 1) ? gdr2::order_bytes(num_seqs) : 0;
     return GDR2_OK;
 }
 
@@ -82,6 +84,7 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     st = gdr2_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, dtype, &need);
     if (st != GDR2_OK) return st;
     if (need > 0 && (!workspace || workspace_bytes < need)) return GDR2_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return GDR2_ERR_INVALID_ARG;
     if (num_seqs == 0) return GDR2_OK;
 
     gdr2::ChunkArgs a;
@@ -89,11 +92,19 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     a.log_alpha = log_alpha;
     a.init_state = init_state;
     a.cu_seqlens = cu_seqlens;
+    a.order = nullptr;
     a.o = o;
     a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.num_seqs = num_seqs;
     a.bf16 = dtype == GDR2_BF16;
-    cudaError_t e = gdr2::chunk_tc_supported(a) ? gdr2::launch_chunk_tc(a, (cudaStream_t)stream)
+    cudaError_t e = cudaSuccess;
+    if (cu_seqlens && num_seqs > 1) {
+        a.order = static_cast<const int32_t *>(workspace);
+        e = gdr2::launch_order_by_length(cu_seqlens, num_seqs, static_cast<int32_t *>(workspace),
+                                         (cudaStream_t)stream);
+        if (e != cudaSuccess) return GDR2_ERR_CUDA;
+    }
+    e = gdr2::chunk_tc_supported(a) ? gdr2::launch_chunk_tc(a, (cudaStream_t)stream)
                                                 : gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }

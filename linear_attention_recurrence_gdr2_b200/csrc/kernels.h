@@ -20,6 +20,7 @@ struct ChunkArgs {
     const float *log_alpha;
     const float *init_state;   // may be null
     const int32_t *cu_seqlens; // may be null
+    const int32_t *order;      // may be null: processing order of the sequences
     void *o;
     float *final_state;        // may be null
     int64_t B, T, H, dk, dv, num_seqs;
@@ -27,6 +28,12 @@ struct ChunkArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// Longest-first sequence order for packed batches (see order.cu).
+constexpr int kMaxSortSeqs = 16384;
+size_t order_bytes(int64_t num_seqs);
+cudaError_t launch_order_by_length(const int32_t *cu_seqlens, int64_t num_seqs, int32_t *order,
+                                   cudaStream_t stream);
 
 // fp32 CUDA-core chunk forward (any dtype; the fp32 path of the library).
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);

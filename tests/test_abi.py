@@ -109,6 +109,15 @@ def test_recurrent_step_rejects_bad_arguments(over, expect):
     assert _step(**over) == expect
 
 
+def test_packed_batch_needs_workspace():
+    need = gdr2.workspace_size(1, 1000, 4, 128, 128, 3, gdr2.GDR2_BF16)
+    assert need >= 3 * 4 and need % 256 == 0
+    assert gdr2.workspace_size(2, 1000, 4, 128, 128, 2, gdr2.GDR2_BF16) == 0
+    assert _chunk(B=1, N=3, cu=FAKE) == WORKSPACE
+    assert _chunk(B=1, N=3, cu=FAKE, ws=FAKE, wsb=need - 1) == WORKSPACE
+    assert _chunk(B=1, N=3, cu=FAKE, ws=FAKE + 8, wsb=need) == INVALID  # misaligned workspace
+
+
 def test_empty_problems_return_ok_without_launch():
     assert _chunk(B=0, N=0, q=None, o=None) == OK
     assert _chunk(B=1, T=0, N=0, cu=FAKE) == OK

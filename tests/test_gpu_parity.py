@@ -72,6 +72,21 @@ def test_chunk_varlen_small(cuda_device, d, dtype):
     check_full(inp, cuda_device, f"varlen d={d} {dtype}")
 
 
+def test_chunk_varlen_many_sequences(cuda_device):
+    """300 packed sequences (lengths 0..200, ties included): exercises the
+    longest-first ordering with a non-power-of-two count."""
+    lengths = np.random.default_rng(12).integers(0, 201, size=300)
+    inp = gen.make_inputs(1, 0, 2, 128, 128, "bf16", seed=12, init_std=0.05, lengths=lengths)
+    check_full(inp, cuda_device, "varlen 300 seqs")
+
+
+def test_chunk_varlen_above_sort_limit(cuda_device):
+    """More sequences than the on-device sort handles: identity order."""
+    lengths = np.random.default_rng(13).integers(0, 4, size=16400)
+    inp = gen.make_inputs(1, 0, 1, 64, 64, "fp32", seed=13, init_std=0.05, lengths=lengths)
+    check_full(inp, cuda_device, "varlen 16400 seqs")
+
+
 def test_chunk_zero_initial_state_and_no_final_state(cuda_device):
     inp = gen.make_inputs(1, 100, 2, 128, 128, "bf16", seed=3)
     o, sf = run_chunk(inp, cuda_device, final=False)

@@ -140,6 +140,38 @@ gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
                                           size_t *bytes);
 
 /*
+ * gdr2_chunk_fwd_noalloc -- gdr2_chunk_fwd for callers that cannot allocate.
+ *
+ * (An addition of this library; the pages have no counterpart.) Some callers
+ * cannot give the library scratch memory: code that is handed only its input
+ * and output buffers by a host framework with no way to ask for more, or
+ * deployments that reserve all device memory up front and must not call
+ * cudaMalloc on the hot path (which can also stall other work on the device).
+ * This entry point takes the same arguments as gdr2_chunk_fwd minus the
+ * workspace and allocates nothing: the one piece of scratch the chunk forward
+ * uses (the longest-first order of a packed batch, 4 bytes per sequence)
+ * lives in a fixed 64 KiB array inside the library, held on every GPU that
+ * loads the library until the process exits.
+ *   - Limit: a packed batch (cu_seqlens, num_seqs > 1) may hold at most 16384
+ *     sequences; larger ones return GDR2_ERR_UNSUPPORTED before any launch.
+ *     Fixed-length batches use no scratch and have no extra limit.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; each call rewrites every entry it reads, so nothing has to be
+ *     cleared, but calls that overlap on the GPU (unordered streams) race on
+ *     it and must be serialised by the caller.
+ * Results are identical to gdr2_chunk_fwd on the same inputs.
+ */
+gdr2_status gdr2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const void *b, const void *w,
+                                   const float *init_state, const int32_t *cu_seqlens,
+                                   int64_t B, int64_t T, int64_t H, int64_t d_k,
+                                   int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                                   void *o, float *final_state, void *stream);
+
+/*
  * gdr2_recurrent_step -- one decode step for N independent sequences.
  *
  * For every sequence n and head h, with the state updated IN PLACE:

@@ -63,6 +63,11 @@ def lib() -> ctypes.CDLL:
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                 _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
                 _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            L.gdr2_chunk_fwd_noalloc.restype = ctypes.c_int
+            L.gdr2_chunk_fwd_noalloc.argtypes = [
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
+                _vp, _vp, _vp]
             L.gdr2_check_device_error.restype = ctypes.c_int
             L.gdr2_check_device_error.argtypes = [_vp]
             L.gdr2_recurrent_step.restype = ctypes.c_int
@@ -178,6 +183,35 @@ def chunk_fwd(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None, *,
         _ptr(workspace), ws_bytes, _stream_handle(stream))
     if st != GDR2_OK:
         raise GDR2Error("gdr2_chunk_fwd", st)
+    return o, final_state
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None, *,
+                      o, final_state=None, stream=None):
+    """gdr2_chunk_fwd_noalloc: the chunk forward with caller-provided outputs
+    and no workspace (for callers that cannot allocate; see gdr2.h). `o` (and
+    `final_state`, if wanted) must be preallocated; nothing is allocated here."""
+    import torch
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("k", k, dk), ("b", b, dk), ("v", v, dv), ("w", w, dv)):
+        _check(t, name, (B, T, H, d), dt, dev)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    N = cu_seqlens.shape[0] - 1 if cu_seqlens is not None else B
+    _check(o, "o", (B, T, H, dv), dt, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (N, H, dk, dv), torch.float32, dev)
+    if final_state is not None:
+        _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
+    st = lib().gdr2_chunk_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(init_state),
+        _ptr(cu_seqlens), B, T, H, dk, dv, N, code, _ptr(o), _ptr(final_state),
+        _stream_handle(stream))
+    if st != GDR2_OK:
+        raise GDR2Error("gdr2_chunk_fwd_noalloc", st)
     return o, final_state
 
 

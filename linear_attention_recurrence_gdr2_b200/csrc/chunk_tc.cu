@@ -80,9 +80,9 @@ constexpr uint64_t kWaitNs = 1000000000ull;  // one second per wait
 // ---- shared memory map (bytes from the 1024-aligned base) ----------------
 constexpr uint32_t kEQ0 = 0;             // per 64-channel block kb: [Em -> -W 8K | Qm 8K]
 constexpr uint32_t kEQ1 = 32768;
-constexpr uint32_t kKB0 = 65536;         // [P 8K | Km kb0 8K | Km kb1 8K]
+constexpr uint32_t kKB0 = 65536;         // [P^T 8K | Km kb0 8K | Km kb1 8K]
 constexpr uint32_t kKB1 = 90112;
-constexpr uint32_t kKmOff = 8192;        // Km after the P block
+constexpr uint32_t kKmOff = 8192;        // Km after the P^T block
 constexpr uint32_t kZB0 = 114688;        // v -> Z: [dv block 0 8K][dv block 1 8K]
 constexpr uint32_t kZB1 = 131072;
 constexpr uint32_t kTB = 147456;         // T bf16, 64 rows x 128 B
@@ -108,8 +108,9 @@ enum {
 constexpr uint32_t kTmU = 0;         // U^T fp32, 64      } one N=128 accumulator
 constexpr uint32_t kTmO = 64;        // O^T fp32, 64      }        } one N=192
 constexpr uint32_t kTmMaster = 128;  // state (transposed) fp32, 128 } accumulator
-constexpr uint32_t kTmAP = 256;      // [A; P] fp32, 64
-constexpr uint32_t kTmW = 320;       // W^T fp32, 64
+constexpr uint32_t kTmX = 256;       // 128 columns shared by two M=64 accumulators:
+                                     //   lanes 0-15 of each quarter: [A^T | P^T] (rows s)
+                                     //   lanes 16-31 of each quarter: W (rows r)
 constexpr uint32_t kTmSB = 384;      // Sm^T bf16 pairs, 64 words
 constexpr uint32_t kTmUB = 448;      // U^T bf16 pairs, 32 words
 
@@ -350,8 +351,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     } else if (warp == 1) {
         // ---------------- MMA issuer for the prep pipeline --------------------
         if (lane == 0) {
-            const uint32_t i_ap = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t i_w = idesc_bf16_f32(128, 64, true, false);
+            const uint32_t i_ap = idesc_bf16_f32(64, 128, false, false);
+            const uint32_t i_w = idesc_bf16_f32(64, 128, false, true);
+            const uint32_t i_u = idesc_bf16_f32(128, 64, true, false);
             for (int cp = 0; cp < nc; ++cp) {
                 const int s = cp & 1;
                 const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
@@ -359,28 +361,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 if (!wait_bar(&bars[B_PREP], cp & 1, abort_flag, 12)) break;
                 if (cp >= 1 && !wait_bar(&bars[B_AFREE], (cp - 1) & 1, abort_flag, 13)) break;
                 tc_fence_after();
-                // [A; P] = [Em; Qm] Km^T
+                // [A^T | P^T] = Km [Em; Qm]^T   (M = 64 rows s, N = 128, lanes 0-15)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tb + kTmAP, a, b, i_ap, kk > 0);
+                    const uint64_t a = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tb + kTmX, a, b, i_ap, kk > 0);
                 }
                 tc_commit(&bars[B_AP]);
                 GDR2_TRACE_AT(cp, 2);
                 if (!wait_bar(&bars[B_T], cp & 1, abort_flag, 14)) break;
-                if (!wait_bar(&bars[B_ZREADY0 + s], (cp >> 1) & 1, abort_flag, 15)) break;
+                // P^T read out of the shared columns (implies Z is ready): the W
+                // accumulator below shares those TMEM columns (other lanes)
+                if (!wait_bar(&bars[B_PREADY0 + s], (cp >> 1) & 1, abort_flag, 15)) break;
                 // the single U region is free once the epilogue has read chunk cp-1's U
                 if (cp >= 1 && !wait_bar(&bars[B_UCONV], (cp - 1) & 1, abort_flag, 16)) break;
                 tc_fence_after();
-                // W^T = Em^T T^T, U0^T = Z^T T^T
+                // W = T Em (M = 64 rows r, N = 128, lanes 16-31); U0^T = Z^T T^T (M = 128)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t at = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
+                    const uint64_t be = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
+                    mma_ss(tb + kTmX + (16u << 16), at, be, i_w, kk > 0);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bt = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
-                    const uint64_t ae = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
                     const uint64_t az = smem_desc_sw128(sbase + (s ? kZB1 : kZB0) + kk * 2048, 8192, 1024);
-                    mma_ss(tb + kTmW, ae, bt, i_w, kk > 0);
-                    mma_ss(tb + kTmU, az, bt, i_w, kk > 0);
+                    mma_ss(tb + kTmU, az, bt, i_u, kk > 0);
                 }
                 tc_commit(&bars[B_WDONE]);
                 GDR2_TRACE_AT(cp, 3);
@@ -396,8 +404,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         // ---------------- MMA issuer for the state chain -----------------------
         if (lane == 0) {
             const uint32_t i_uo = idesc_bf16_f32(128, 128, false, false);
-            const uint32_t i_op = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t i_mk = idesc_bf16_f32(128, 128, false, true);
+            const uint32_t i_os = idesc_bf16_f32(128, 192, false, true);
             for (int cc = 0; cc < nc; ++cc) {
                 const int s = cc & 1;
                 const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
@@ -418,16 +425,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 if (!wait_bar(&bars[B_PREADY0 + s], (cc >> 1) & 1, abort_flag, 25)) break;
                 GDR2_TRACE_AT(cc, 6);
                 tc_fence_after();
-                // O^T += U^T P^T (B = P, K-major), M^T += U^T Km (B = Km, MN-major)
+                // [O^T | M^T] += U^T [P^T | Km]   (N = 192, B MN-major: P^T atom, two Km atoms)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t b = smem_desc_sw128(kbs + kk * 32, 16, 1024);
-                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, b, i_op, 1);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t b = smem_desc_sw128(kbs + kKmOff + kk * 2048, 8192, 1024);
-                    mma_ts(tb + kTmMaster, tb + kTmUB + kk * 8, b, i_mk, 1);
+                    const uint64_t b = smem_desc_sw128(kbs + kk * 2048, 8192, 1024);
+                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, b, i_os, 1);
                 }
                 tc_commit(&bars[B_SDONE]);
                 GDR2_TRACE_AT(cc, 5);
@@ -587,24 +589,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_arrive(&bars[B_ZREADY0 + s]);
             }
 
-            // P = tril(Qm Km^T) from TMEM lanes 64-127 -> K-major rows before Km
+            // P^T[s][r] = P[r][s] (kept for s <= r) from the M=64 accumulator: lane
+            // i < 16 of warp pw holds row s = 16 pw + i -> MN-major rows before Km
             if (!group_and(kBarPrepA, wait_bar(&bars[B_AP], c & 1, abort_flag, 6))) break;
             if (tp == 0) GDR2_TRACE_AT(c, 13);
             tc_fence_after();
-            if (pw >= 2) {
-                const uint32_t taddr = tb + kTmAP + ((uint32_t)(32 * pw) << 16);
+            {
+                const uint32_t taddr = tb + kTmX + 64 + ((uint32_t)(32 * pw) << 16);
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
                 tc_wait_ld();
-                const int r = 32 * (pw - 2) + lane;
-                float x[64];
+                if (lane < 16) {
+                    const int srow = 16 * pw + lane;
+                    float x[64];
 #pragma unroll
-                for (int j2 = 0; j2 < 32; ++j2) {
-                    x[j2] = j2 <= r ? __uint_as_float(v0[j2]) : 0.f;
-                    x[32 + j2] = 32 + j2 <= r ? __uint_as_float(v1[j2]) : 0.f;
+                    for (int j2 = 0; j2 < 32; ++j2) {
+                        x[j2] = j2 >= srow ? __uint_as_float(v0[j2]) : 0.f;
+                        x[32 + j2] = 32 + j2 >= srow ? __uint_as_float(v1[j2]) : 0.f;
+                    }
+                    store_row_bf16_sw128(smem + (s ? kKB1 : kKB0), srow, x);
                 }
-                store_row_bf16_sw128(smem + (s ? kKB1 : kKB0), r, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -628,22 +633,42 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (!group_and(kBarPrepB, wait_bar(&bars[B_AP], c & 1, abort_flag, 7))) break;
             if (tp == 0) GDR2_TRACE_AT(c, 15);
             tc_fence_after();
-            if (pw < 2) {  // A rows (TMEM lanes 0-63) -> A^T[s][r] for s < r
-                const uint32_t taddr = tb + kTmAP + ((uint32_t)(32 * pw) << 16);
+            {   // A^T rows from the M=64 accumulator (lane i < 16 of warp pw: row s = 16 pw + i):
+                // A^T[s][r] = A[r][s], kept for r > s
+                const uint32_t taddr = tb + kTmX + ((uint32_t)(32 * pw) << 16);
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
                 tc_wait_ld();
-                const int r = 32 * pw + lane;
+                if (lane < 16) {
+                    const int srow = 16 * pw + lane;
+                    float *row = sA + srow * kLD;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sA[j * kLD + r] = j < r ? __uint_as_float(v0[j]) : 0.f;
-                    sA[(32 + j) * kLD + r] = 32 + j < r ? __uint_as_float(v1[j]) : 0.f;
+                    for (int q = 0; q < 8; ++q) {
+                        float4 a0, a1;
+                        a0.x = 4 * q + 0 > srow ? __uint_as_float(v0[4 * q + 0]) : 0.f;
+                        a0.y = 4 * q + 1 > srow ? __uint_as_float(v0[4 * q + 1]) : 0.f;
+                        a0.z = 4 * q + 2 > srow ? __uint_as_float(v0[4 * q + 2]) : 0.f;
+                        a0.w = 4 * q + 3 > srow ? __uint_as_float(v0[4 * q + 3]) : 0.f;
+                        a1.x = 32 + 4 * q + 0 > srow ? __uint_as_float(v1[4 * q + 0]) : 0.f;
+                        a1.y = 32 + 4 * q + 1 > srow ? __uint_as_float(v1[4 * q + 1]) : 0.f;
+                        a1.z = 32 + 4 * q + 2 > srow ? __uint_as_float(v1[4 * q + 2]) : 0.f;
+                        a1.w = 32 + 4 * q + 3 > srow ? __uint_as_float(v1[4 * q + 3]) : 0.f;
+                        *reinterpret_cast<float4 *>(row + 4 * q) = a0;
+                        *reinterpret_cast<float4 *>(row + 32 + 4 * q) = a1;
+                    }
                 }
             }
             tc_fence_before();
             named_bar_sync(kBarPrepB, 128);
-            if (tp == 0) { GDR2_TRACE_AT(c, 25); mbar_arrive(&bars[B_AFREE]); }
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 25);
+                // lanes 0-15 of the shared columns may now take the next [A^T | P^T]
+                // (prep A has read its P^T: that precedes PREP of the next chunk).
+                // The W readout below still loads all 32 lanes of each quarter,
+                // but it only uses lanes 16-31, which that MMA does not write.
+                mbar_arrive(&bars[B_AFREE]);
+            }
 
             // T = (I + A)^{-1} by doubling on 16-row blocks (A held transposed,
             // sA = A^T; T in sT, both fp32 with row pitch kLD):
@@ -747,21 +772,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (!group_and(kBarPrepB, wait_bar(&bars[B_WDONE], c & 1, abort_flag, 8))) break;
             if (tp == 0) GDR2_TRACE_AT(c, 17);
             tc_fence_after();
-            {
-                const uint32_t taddr = tb + kTmW + ((uint32_t)(32 * pw) << 16);
-                uint32_t v0[32], v1[32];
-                tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
-                tc_wait_ld();
-                const int ch = 32 * pw + lane;
-                unsigned char *wt = smem + (s ? kEQ1 : kEQ0) + (ch >> 6) * 16384;
-                const uint32_t cb = 2 * (ch & 63);
+            {   // W rows from the M=64 accumulator (lane 16 + i of warp pw: row r = 16 pw + i)
+                // -> -W, K-major, over the Em half of the slot (two 64-channel blocks)
+                const uint32_t taddr = tb + kTmX + ((uint32_t)(32 * pw) << 16);
+                const int rrow = 16 * pw + (lane & 15);
+#pragma unroll 1
+                for (int hb = 0; hb < 2; ++hb) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(taddr + 64 * hb, v0);
+                    tmem_ld32(taddr + 64 * hb + 32, v1);
+                    tc_wait_ld();
+                    if (lane >= 16) {
+                        float x[64];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(j, cb)) =
-                        __float2bfloat16_rn(-__uint_as_float(v0[j]));
-                    *reinterpret_cast<__nv_bfloat16 *>(wt + sw128_offset(32 + j, cb)) =
-                        __float2bfloat16_rn(-__uint_as_float(v1[j]));
+                        for (int j2 = 0; j2 < 32; ++j2) {
+                            x[j2] = -__uint_as_float(v0[j2]);
+                            x[32 + j2] = -__uint_as_float(v1[j2]);
+                        }
+                        store_row_bf16_sw128(smem + (s ? kEQ1 : kEQ0) + hb * 16384, rrow, x);
+                    }
                 }
             }
             fence_proxy_async_smem();

@@ -65,6 +65,22 @@ def workload(name: str):
     raise ValueError(name)
 
 
+def measured_traffic():
+    """DRAM bytes per chunk-forward launch from the committed ncu capture
+    (profiles/traffic.json), or None once the kernel source has changed since
+    the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except (OSError, KeyError, ValueError):
+        return None
+    return int(t["bytes_per_launch"]) if sha == t["source_sha256_16"] else None
+
+
 def chunk_bytes(inp) -> int:
     """Algorithmic HBM bytes of one chunk-forward launch: every input read
     once, o written once, initial states read once (if given), final states
@@ -370,7 +386,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent sequences per GPU)",
                    "l2": "inputs larger than L2 (no flush)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
+                     "frac": achieved / hbm_peak,
+                     "traffic": measured_traffic() if args.workload == "prefill" else None,
                      "kernel": "chunk forward", "bytes_per_launch": nbytes,
                      "us_per_launch": kern_ms * 1e3, "peak_source": peak_src},
         "decode": {"workload": "N=256 x H=16, d=128, fp32 state, bf16 tokens",

@@ -1037,6 +1037,32 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+namespace {
+// One CTA waiting on a barrier that nothing arrives on, through the kernel's
+// bounded wait with a caller-chosen limit (failure-detection self-test).
+__global__ void wait_selftest_kernel(uint64_t timeout_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        WaitGuard g{globaltimer_ns() + timeout_ns, &abort_flag, &g_chunk_tc_error};
+        mbar_wait(&bar, 0, g, 31);
+    }
+}
+}  // namespace
+
+cudaError_t chunk_tc_wait_selftest(uint32_t timeout_us, cudaStream_t stream)
+{
+    wait_selftest_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 1000ull);
+    return cudaGetLastError();
+}
+
 cudaError_t chunk_tc_read_and_clear_error(int *code)
 {
     int zero = 0;

@@ -1,6 +1,7 @@
 // C ABI of the Gated Delta Rule-2 library: argument validation and dispatch.
 // Declarations and the full contract are in include/gdr2.h.
 #include "../../include/gdr2.h"
+#include "../../include/gdr2_testing.h"
 #include "kernels.h"
 
 #include <cuda_runtime.h>
@@ -141,6 +142,13 @@ gdr2_status gdr2_check_device_error(void *stream)
     int code = 0;
     if (gdr2::chunk_tc_read_and_clear_error(&code) != cudaSuccess) return GDR2_ERR_CUDA;
     return code ? GDR2_ERR_DEVICE_TIMEOUT : GDR2_OK;
+}
+
+gdr2_status gdr2_selftest_bounded_wait(uint32_t timeout_us, void *stream)
+{
+    if (timeout_us == 0 || timeout_us > 2000000u) return GDR2_ERR_INVALID_ARG;
+    return gdr2::chunk_tc_wait_selftest(timeout_us, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK
+                                                                                         : GDR2_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -45,4 +45,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 // Reads and clears the tensor-core kernel's device error word (synchronous).
 cudaError_t chunk_tc_read_and_clear_error(int *code);
 
+// Failure-detection self-test: one bounded wait that runs out after timeout_us.
+cudaError_t chunk_tc_wait_selftest(uint32_t timeout_us, cudaStream_t stream);
+
 }  // namespace gdr2

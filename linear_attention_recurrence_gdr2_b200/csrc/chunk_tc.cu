@@ -1,5 +1,6 @@
 // Chunkwise forward of Gated Delta Rule-2 for bf16 inputs, d_k = d_v = 128,
-// on the sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA).
+// on the sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA), one
+// cluster of two CTAs per (sequence, head).
 //
 // Chunk form (C = 64; "Chunkwise training and gate-aware backward" section
 // of the ainews.random.gg article on Gated DeltaNet-2). Per chunk with entry
@@ -16,35 +17,39 @@
 // Sm = Diag(e^{g_31}) S0, which makes Qm Sm = Qbar S0 and (T Em) Sm = W S0,
 // and the state update becomes S_C = Diag(e^{g_C - g_31}) (Sm + Km^T U).
 //
-// One CTA owns one (sequence, head) and walks its chunks in order. Everything
-// is computed transposed so that the value dimension (128) sits on the MMA's
-// M axis and on the 128 TMEM lanes (P = tril(Qm Km^T), M = the TMEM state):
-//     [A; P]        = [Em; Qm] Km^T                 M=128 N=64  K=128
-//     W^T, U0^T     = Em^T T^T, Z^T T^T             M=128 N=64  K=64 (x2)
-//     [U^T | O^T]  += Sm^T [-W; Qm]^T               M=128 N=128 K=128, A in TMEM
-//     [O^T | M^T]  += U^T [P^T | Km]                M=128 N=192 K=64,  A in TMEM
-// Merging the products that share an A operand into one wide-N chain keeps
-// the number of tcgen05.mma instructions per chunk at 28 (each costs a fixed
-// issue time whatever its N). -W is written K-major over Em (dead by then) so
-// that it sits right before Qm; P^T is written MN-major right before Km; the
-// O columns sit between U and the state in TMEM.
-// The fp32 state lives in TMEM (as M = Diag(e^{g_31}) S plus the chunk's
-// update); once per chunk the epilogue scales it by e^{g_C - g_31 + g'_31}
-// (g'_31: the next chunk's half sum) and writes its bf16 copy back to TMEM as
-// the next chunk's MMA operand.
+// Work split. Only the state chain is serial across chunks; everything that
+// depends on one chunk's inputs alone runs ahead of it on a second SM:
+//   helper CTA (cluster rank 1), per chunk:
+//     decay sums and factors Qm, Km, Em (in place over the q, k, b tiles),
+//     [A^T | P^T] = Km [Em; Qm]^T       M=64  N=128 K=128 (tcgen05),
+//     T = (I + A)^{-1} (tf32 mma.sync doubling) as bf16,
+//     and bulk copies of Em, Qm, Km, P^T, T and the half sums into the main
+//     CTA's shared memory (distributed shared memory inside the cluster);
+//   main CTA (cluster rank 0), per chunk:
+//     Z = w . v; W = T Em (two M=64 halves); U0^T = Z^T T^T;
+//     [U^T | O^T]  += Sm^T [-W; Qm]^T   M=128 N=128 K=128, A in TMEM
+//     [O^T | M^T]  += U^T [P^T | Km]    M=128 N=192 K=64,  A in TMEM
+//     and the epilogue (U^T to bf16, o stores, state scaling, final state).
+// Everything is computed transposed so that the value dimension (128) sits
+// on the MMA's M axis and on the 128 TMEM lanes. The fp32 state lives in the
+// main CTA's TMEM (as M = Diag(e^{g_31}) S plus the chunk's update); once per
+// chunk the epilogue scales it by e^{g_C - g_31 + g'_31} (g'_31: the next
+// chunk's half sum) and writes its bf16 copy back to TMEM as the next chunk's
+// MMA operand. Both CTAs double-buffer their chunk slots; the main CTA tells
+// the helper when a slot has been consumed (remote mbarrier arrives), the
+// helper's copies complete on the main CTA's barriers.
 //
-// Warp roles (16 warps; the first warpgroup gives registers to the others):
-//   0      TMA producer of q, k, b tiles (double-buffered slots)
-//   1      tcgen05.mma issuer of the prep pipeline ([A;P], W^T, U0^T)
-//   2      TMEM allocator; TMA producer of v tiles, L2 prefetch of w
-//   3      tcgen05.mma issuer of the state chain
-//   4..7   prep A: cumulative decay, decay-absorbed factors, Z, P^T
-//   8..11  prep B: (I + A)^{-1}, -W
-//   12..15 epilogue: U^T to bf16, o stores, state scaling, final state
-// The two prep warpgroups work on consecutive chunks concurrently, and both
-// run ahead of the state chain. Every wait is bounded: after about a second
-// without progress the CTA records the site in the device error word and
-// winds down (drains its TMA loads and MMAs, frees TMEM, returns).
+// Warp roles (16 warps per CTA; the first warpgroup gives registers away):
+//   main:   0 v TMA producer, w L2 prefetch, slot-free relay
+//           1 tcgen05.mma issuer: W, U0      2 TMEM allocator, copy-landed relay
+//           3 tcgen05.mma issuer: state chain
+//           4..7 Z      8..11 -W from TMEM      12..15 epilogue
+//   helper: 0 q, k, b TMA producer           1 tcgen05.mma issuer: [A^T | P^T]
+//           2 TMEM allocator                  4..11 decay factors, P^T
+//           12..15 (I + A)^{-1}
+// Every wait is bounded: after about a second without progress the CTA
+// records the site in the device error word, tells its peer to wind down,
+// drains its own TMA loads and MMAs, frees TMEM, and returns.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -65,8 +70,15 @@ __device__ unsigned long long *g_chunk_tc_trace;
         if (blockIdx.x < 4 && g_chunk_tc_trace && (chunk) < 1024)                          \
             g_chunk_tc_trace[((size_t)blockIdx.x * 1024 + (chunk)) * 32 + (ev)] = clock64(); \
     } while (0)
+// [CTA][start ns, end ns, SM id] for every CTA (buffer sized by the driver)
+__device__ unsigned long long *g_chunk_tc_span;
+#define GDR2_SPAN_AT(slot, value)                                                          \
+    do {                                                                                   \
+        if (g_chunk_tc_span) g_chunk_tc_span[(size_t)blockIdx.x * 3 + (slot)] = (value);   \
+    } while (0)
 #else
 #define GDR2_TRACE_AT(chunk, ev) do { } while (0)
+#define GDR2_SPAN_AT(slot, value) do { } while (0)
 #endif
 
 namespace {
@@ -76,46 +88,64 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kThreadsTC = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;  // one second per wait
+constexpr int kPairs = 2;                     // (sequence, head) units per cluster
 
-// ---- shared memory map (bytes from the 1024-aligned base) ----------------
-constexpr uint32_t kEQ0 = 0;             // per 64-channel block kb: [Em -> -W 8K | Qm 8K]
-constexpr uint32_t kEQ1 = 32768;
-constexpr uint32_t kKB0 = 65536;         // [P^T 8K | Km kb0 8K | Km kb1 8K]
-constexpr uint32_t kKB1 = 90112;
-constexpr uint32_t kKmOff = 8192;        // Km after the P^T block
-constexpr uint32_t kZB0 = 114688;        // v -> Z: [dv block 0 8K][dv block 1 8K]
-constexpr uint32_t kZB1 = 131072;
-constexpr uint32_t kTB = 147456;         // T bf16, 64 rows x 128 B
-constexpr uint32_t kLA = 155648;         // staged log_alpha, fp32 [64][128]
-constexpr int kLD = 68;                  // fp32 scratch row pitch (16-byte aligned rows)
-constexpr uint32_t kSA = 188416;         // fp32 A^T, 64 x kLD
-constexpr uint32_t kST = kSA + 64 * kLD * 4;  // fp32 T, 64 x kLD
-constexpr uint32_t kVEC = kST + 64 * kLD * 4; // half sums: T0[4][128], T1[4][128], f[128]
-constexpr uint32_t kBSUM = kVEC + (8 * 128 + 128) * 4;  // per-row-block log-decay sums [4][128]
-constexpr uint32_t kBAR = kBSUM + 4 * 128 * 4;
-constexpr int kNumBars = 28;
-constexpr uint32_t kMISC = kBAR + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kMISC + 64 + 1024;  // + alignment slack
+// ---- main CTA shared memory (bytes from the 1024-aligned base) -------------
+__host__ __device__ constexpr uint32_t mEQ(int s) { return s ? 32768 : 0; }          // per key block kb: [Em -> -W 8K | Qm 8K]
+__host__ __device__ constexpr uint32_t mKB(int s) { return s ? 90112 : 65536; }      // [P^T 8K | Km kb0 8K | Km kb1 8K]
+constexpr uint32_t kKmOff = 8192;                  // Km after the P^T block
+__host__ __device__ constexpr uint32_t mZ(int s) { return s ? 131072 : 114688; }     // v -> Z: [dv block 0 8K][dv block 1 8K]
+__host__ __device__ constexpr uint32_t mT(int s) { return s ? 155648 : 147456; }     // T bf16, 64 rows x 128 B
+__host__ __device__ constexpr uint32_t mVEC(int s) { return s ? 164864 : 163840; }   // half sums [T0 | T1], fp32 128 + 128
+constexpr uint32_t kM_VECF = 165888;               // state scale factors, fp32 128
+// ---- helper CTA shared memory ----------------------------------------------
+__host__ __device__ constexpr uint32_t hEQ(int s) { return s ? 49152 : 0; }          // [b -> Em | q -> Qm] per key block, then k -> Km
+constexpr uint32_t kH_KmOff = 32768;
+__host__ __device__ constexpr uint32_t hPT(int s) { return s ? 106496 : 98304; }     // P^T bf16 (MN-major operand rows s)
+__host__ __device__ constexpr uint32_t hT(int s) { return s ? 122880 : 114688; }     // T bf16
+constexpr uint32_t kH_LA = 131072;                 // staged log_alpha, fp32 [64][128]
+constexpr int kLD = 68;                            // fp32 scratch row pitch (16-byte aligned rows)
+constexpr uint32_t kH_SA = 163840;                 // fp32 A^T, 64 x kLD
+constexpr uint32_t kH_ST = kH_SA + 64 * kLD * 4;   // fp32 T, 64 x kLD
+__host__ __device__ constexpr uint32_t hVEC(int s) { return s ? kH_ST + 64 * kLD * 4 + 1024 : kH_ST + 64 * kLD * 4; }
+constexpr uint32_t kH_BSUM = hVEC(1) + 1024;     // per-row-block log-decay sums [8][128]
+// ---- both ------------------------------------------------------------------
+constexpr uint32_t kBAR = kH_BSUM + 8 * 128 * 4;   // same offset in both CTAs
+constexpr int kNumBars = 32;
+constexpr uint32_t kMISC = kBAR + kNumBars * 8;    // TMEM slot, abort flag, copy counters
+constexpr uint32_t kSmemBytes = kMISC + 64 + 1024; // + alignment slack
+static_assert(kM_VECF + 512 <= kBAR, "main shared-memory map overlaps the barriers");
+static_assert(kSmemBytes <= 232448, "shared memory above the per-CTA limit");
 
-// barrier indices
+constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
+
+// barriers of the main CTA
 enum {
-    B_FULL0 = 0, B_FULL1, B_SLOTFREE0, B_SLOTFREE1, B_VFULL0, B_VFULL1, B_VFREE0, B_VFREE1,
-    B_LAFULL, B_PREP, B_VEC0, B_VEC1, B_AP, B_AFREE, B_ZREADY0, B_ZREADY1, B_T, B_WDONE, B_WREADY0,
-    B_WREADY1, B_PREADY0, B_PREADY1, B_SREADY, B_UDONE, B_UCONV, B_SDONE, B_DRAIN, B_DRAIN2
+    M_F0 = 0, M_F1, M_P0, M_P1, M_T0, M_T1, M_VFULL0, M_VFULL1, M_VFREE0, M_VFREE1, M_ZREADY0, M_ZREADY1,
+    M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY, M_UDONE, M_UCONV, M_SDONE, M_SLOTFREE0,
+    M_SLOTFREE1, M_DRAIN, M_DRAIN2, M_NUM
 };
+// barriers of the helper CTA
+enum {
+    H_FULL0 = 0, H_FULL1, H_SLOTFREE0, H_SLOTFREE1, H_LAFULL, H_FDONE, H_AP0, H_AP1, H_XFREE0,
+    H_XFREE1, H_MFREE0, H_MFREE1, H_TFREE0, H_TFREE1, H_DRAIN, H_NUM
+};
+static_assert(M_NUM <= kNumBars && H_NUM <= kNumBars, "barrier area too small");
 
-// ---- TMEM column map (512 columns allocated) -------------------------------
+// ---- TMEM column maps -------------------------------------------------------
+// main (512 columns allocated)
 constexpr uint32_t kTmU = 0;         // U^T fp32, 64      } one N=128 accumulator
 constexpr uint32_t kTmO = 64;        // O^T fp32, 64      }        } one N=192
 constexpr uint32_t kTmMaster = 128;  // state (transposed) fp32, 128 } accumulator
-constexpr uint32_t kTmX = 256;       // 128 columns shared by two M=64 accumulators:
-                                     //   lanes 0-15 of each quarter: [A^T | P^T] (rows s)
-                                     //   lanes 16-31 of each quarter: W (rows r)
-constexpr uint32_t kTmSB = 384;      // Sm^T bf16 pairs, 64 words
-constexpr uint32_t kTmUB = 448;      // U^T bf16 pairs, 32 words
+constexpr uint32_t kTmW = 256;       // W (M=64): lanes 0-15 of each quarter key channels 0-63,
+                                     //           lanes 16-31 key channels 64-127; 64 columns
+constexpr uint32_t kTmSB = 320;      // Sm^T bf16 pairs, 64 words
+constexpr uint32_t kTmUB = 384;      // U^T bf16 pairs, 32 words
+// helper (256 columns): [A^T | P^T] (M=64, lanes 0-15 of each quarter) for slot s at 128 s
 
-// group (named) barriers
-constexpr uint32_t kBarPrepA = 1, kBarEpi = 2, kBarPrepB = 3;
+// group (named) barriers, per CTA
+constexpr uint32_t kBarZ = 1, kBarEpi = 2, kBarW = 3;   // main
+constexpr uint32_t kBarPrepA = 1, kBarPrepB = 3;        // helper
 
 struct TcParams {
     const float *la;
@@ -125,46 +155,39 @@ struct TcParams {
     const int32_t *order;
     __nv_bfloat16 *o;
     float *final_state;
-    int64_t T, H;
+    int64_t T, H, units;
 };
 
+// Bounded wait on a barrier of this CTA (CTA-scope acquire: the peer's
+// arrives only signal, and its data arrives by bulk copies that complete on
+// this CTA's barriers). A wait that fails also raises the peer CTA's abort
+// flag, so that the whole cluster winds down.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         int site) {
+                                         uint32_t peer_abort, int site) {
     WaitGuard g{globaltimer_ns() + kWaitNs, abort_flag, &g_chunk_tc_error};
-    return mbar_wait(bar, parity, g, site);
+    const bool ok = mbar_wait(bar, parity, g, site);
+    if (!ok) st_cluster_u32(peer_abort, 1u);
+    return ok;
 }
 
-// Barrier over a 128-thread group that also ANDs one predicate across it, so
+// Bounded wait used only while winding down (never raises the abort flag).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int site) {
+    volatile int dummy = 0;
+    WaitGuard g{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+    mbar_wait(bar, parity, g, site);
+}
+
+// Barrier over an n-thread group that also ANDs one predicate across it, so
 // every thread of the group takes the same continue / abort decision.
-__device__ __forceinline__ bool group_and(uint32_t id, bool v) {
+__device__ __forceinline__ bool group_and(uint32_t id, uint32_t n, bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pi, po;\n\t"
         "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.and.pred po, %2, 128, pi;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
         "selp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r) : "r"((uint32_t)v), "r"(id) : "memory");
+        : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
     return r != 0;
-}
-
-// Bounded spin on a barrier phase without suspending (for the MMA issuers,
-// whose reaction time is on the chunk-to-chunk path).
-__device__ __forceinline__ bool spin_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         int site) {
-    uint64_t deadline = 0;
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 1023u) == 1023u) {
-            if (*abort_flag) return false;
-            const uint64_t now = globaltimer_ns();
-            if (deadline == 0) deadline = now + kWaitNs;
-            else if (now > deadline) {
-                *abort_flag = 1;
-                atomicCAS(&g_chunk_tc_error, 0, 0x100 | site);
-                return false;
-            }
-        }
-    }
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
@@ -241,177 +264,187 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Align to 1024 B by offsetting the __shared__ array itself (not through an
     // integer round trip), so every access below stays a shared-space access.
+    // Both CTAs of the cluster get the same offsets.
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kMISC + 4);
-    float *sA = reinterpret_cast<float *>(smem + kSA);
-    float *sT = reinterpret_cast<float *>(smem + kST);
-    float *vecT0 = reinterpret_cast<float *>(smem + kVEC);         // [4][128]
-    float *vecT1 = vecT0 + 4 * 128;                                 // [4][128]
-    float *vecF = vecT1 + 4 * 128;                                  // [128]
-    float *vecBS = reinterpret_cast<float *>(smem + kBSUM);         // [4][128]
+    uint32_t *copy_count = reinterpret_cast<uint32_t *>(smem + kMISC + 8);  // helper: [F0 F1 P0 P1 T0 T1]
 
+    // Cluster ranks [0, kPairs) are the main CTAs of kPairs units, ranks
+    // [kPairs, 2 kPairs) their helpers (so that CTAs running the same code
+    // share a TPC); unit sub of the cluster is served by ranks sub, kPairs + sub.
+    const uint32_t rank = cluster_ctarank();
+    const bool is_main = rank < (uint32_t)kPairs;
+    const uint32_t peer = is_main ? rank + kPairs : rank - kPairs;
+    const uint32_t peer_abort = mapa_shared(sbase + kMISC + 4, peer);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = prm.H;
-    const int64_t h = blockIdx.x % H;
-    const int64_t n = prm.order ? (int64_t)prm.order[blockIdx.x / H] : (int64_t)(blockIdx.x / H);
-    int64_t t_begin, t_end;
-    if (prm.cu_seqlens) {
-        t_begin = prm.cu_seqlens[n];
-        t_end = prm.cu_seqlens[n + 1];
-    } else {
-        t_begin = n * prm.T;
-        t_end = t_begin + prm.T;
+    const int64_t unit = (int64_t)(blockIdx.x / (2 * kPairs)) * kPairs + (rank % kPairs);
+    const bool valid = unit < prm.units;  // the last cluster may hold a padding pair
+    int64_t h = 0, n = 0, t_begin = 0, t_end = 0;
+    if (valid) {
+        h = unit % H;
+        n = prm.order ? (int64_t)prm.order[unit / H] : (int64_t)(unit / H);
+        if (prm.cu_seqlens) {
+            t_begin = prm.cu_seqlens[n];
+            t_end = prm.cu_seqlens[n + 1];
+        } else {
+            t_begin = n * prm.T;
+            t_end = t_begin + prm.T;
+        }
     }
     const int nc = (int)((t_end - t_begin + 63) / 64);
     const int64_t state_base = (n * H + h) * (int64_t)kD * kD;
 
-    if (nc == 0) {  // empty sequence: the final state is the initial state
-        if (prm.final_state)
+    if (nc == 0) {
+        // empty sequence (both CTAs of the pair are here): the final state is
+        // the initial state; then only the cluster's three barriers are joined
+        if (valid && is_main && prm.final_state)
             for (int i = tid; i < kD * kD; i += kThreadsTC)
                 prm.final_state[state_base + i] = prm.init_state ? prm.init_state[state_base + i] : 0.f;
+        cluster_sync_all();
+        cluster_sync_all();
+        cluster_sync_all();
         return;
     }
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], 1);
+        if (!is_main) {
+            // q, k, b slot: freed by the [A^T | P^T] MMAs and by the main CTA having
+            // received the factors; X columns: freed by both readout groups
+            mbar_init(&bars[H_SLOTFREE0], 2);
+            mbar_init(&bars[H_SLOTFREE1], 2);
+            mbar_init(&bars[H_XFREE0], 2);
+            mbar_init(&bars[H_XFREE1], 2);
+        }
         *abort_flag = 0;
+        for (int i = 0; i < 6; ++i) copy_count[i] = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&map_q); prefetch_tensormap(&map_k); prefetch_tensormap(&map_b);
+        if (is_main) {
+            prefetch_tensormap(&map_v); prefetch_tensormap(&map_w);
+        } else {
+            prefetch_tensormap(&map_q); prefetch_tensormap(&map_k); prefetch_tensormap(&map_b);
+            prefetch_tensormap(&map_la);
+        }
     }
     if (warp == 2) {
-        if (lane == 0) {
-            prefetch_tensormap(&map_v); prefetch_tensormap(&map_la); prefetch_tensormap(&map_w);
-        }
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, is_main ? 512 : 256);
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote access
     tc_fence_after();
     const uint32_t tb = *tmem_slot;
+    if (tid == 0) {
+        GDR2_TRACE_AT(0, 31);  // common time base of the two CTAs
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        GDR2_SPAN_AT(0, globaltimer_ns());
+        GDR2_SPAN_AT(2, smid);
+    }
 
-    // =====================================================================
+    if (is_main) {
+    // =========================================================================
+    //                               main CTA
+    // =========================================================================
     if (warp < 4) {
     setmaxnreg_dec40();
     if (warp == 0) {
-        // ---------------- producer: q, k, b tiles ----------------------------
+        // ------------- v tiles, L2 prefetch of w, slot-free relay -------------
         if (lane == 0) {
-            int issued[2] = {0, 0};
-            for (int c = 0; c < nc; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !wait_bar(&bars[B_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, 1)) break;
-                const int z = (int)(t_begin + 64 * c);
-                unsigned char *eq = smem + (s ? kEQ1 : kEQ0), *kq = smem + (s ? kKB1 : kKB0) + kKmOff;
-                GDR2_TRACE_AT(c, 0);
-                mbar_arrive_expect_tx(&bars[B_FULL0 + s], 3 * 16384);
-                for (int blk = 0; blk < 2; ++blk) {
-                    tma_load_3d(eq + blk * 16384, &map_b, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
-                    tma_load_3d(eq + blk * 16384 + 8192, &map_q, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
-                    tma_load_3d(kq + blk * 8192, &map_k, &bars[B_FULL0 + s], 64 * blk, (int)h, z);
-                }
-                issued[s] = (c >> 1) + 1;
-            }
-            // drain: wait (bounded) for every load issued into each slot
-            for (int s = 0; s < 2; ++s)
-                if (issued[s] > 0) {
-                    volatile int dummy = 0;
-                    WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-                    mbar_wait(&bars[B_FULL0 + s], (issued[s] - 1) & 1, g2, 20);
-                }
-        }
-    } else if (warp == 2) {
-        // ---------------- producer: v tiles, L2 prefetch of w ------------------
-        if (lane == 0) {
+            const uint32_t h_mfree = mapa_shared(smem_u32(&bars[H_MFREE0]), peer);
             tma_prefetch_3d(&map_w, 0, (int)h, (int)t_begin);
-            int vissued[2] = {0, 0};
+            int vissued0 = 0, vissued1 = 0;  // loads issued into each slot
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                if (c >= 2 && !wait_bar(&bars[B_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, 2)) break;
+                if (c >= 2 && !wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
+                    break;
                 const int z = (int)(t_begin + 64 * c);
-                GDR2_TRACE_AT(c, 1);
-                mbar_arrive_expect_tx(&bars[B_VFULL0 + s], 16384);
+                GDR2_TRACE_AT(c, 0);
+                mbar_arrive_expect_tx(&bars[M_VFULL0 + s], 16384);
                 for (int blk = 0; blk < 2; ++blk)
-                    tma_load_3d(smem + (s ? kZB1 : kZB0) + blk * 8192, &map_v, &bars[B_VFULL0 + s], 64 * blk,
-                                (int)h, z);
-                vissued[s] = (c >> 1) + 1;
+                    tma_load_3d(smem + mZ(s) + blk * 8192, &map_v, &bars[M_VFULL0 + s], 64 * blk, (int)h, z);
+                (s ? vissued1 : vissued0) = (c >> 1) + 1;
                 if (c + 1 < nc) tma_prefetch_3d(&map_w, 0, (int)h, z + 64);
-            }
-            for (int s = 0; s < 2; ++s)
-                if (vissued[s] > 0) {
-                    volatile int dummy = 0;
-                    WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-                    mbar_wait(&bars[B_VFULL0 + s], (vissued[s] - 1) & 1, g2, 21);
+                // slot s of chunk c - 2 fully consumed (its last MMA is done):
+                // the helper may copy chunk c into it
+                if (c >= 2) {
+                    if (!wait_bar(&bars[M_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 2)) break;
+                    mbar_remote_arrive(h_mfree + 8 * s);
+                    GDR2_TRACE_AT(c - 2, 15);
                 }
+            }
+            if (vissued0 > 0) drain_wait(&bars[M_VFULL0], (vissued0 - 1) & 1, 20);
+            if (vissued1 > 0) drain_wait(&bars[M_VFULL1], (vissued1 - 1) & 1, 20);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer for the prep pipeline --------------------
+        // ------------- MMA issuer: W = T Em, U0^T = Z^T T^T --------------------
         if (lane == 0) {
-            const uint32_t i_ap = idesc_bf16_f32(64, 128, false, false);
-            const uint32_t i_w = idesc_bf16_f32(64, 128, false, true);
+            const uint32_t i_w = idesc_bf16_f32(64, 64, false, true);
             const uint32_t i_u = idesc_bf16_f32(128, 64, true, false);
-            for (int cp = 0; cp < nc; ++cp) {
-                const int s = cp & 1;
-                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
-                const uint32_t km = sbase + (s ? kKB1 : kKB0) + kKmOff;
-                if (!wait_bar(&bars[B_PREP], cp & 1, abort_flag, 12)) break;
-                if (cp >= 1 && !wait_bar(&bars[B_AFREE], (cp - 1) & 1, abort_flag, 13)) break;
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                const uint32_t eq = sbase + mEQ(s), tt = sbase + mT(s), zz = sbase + mZ(s);
+                if (!wait_bar(&bars[M_F0 + s], (c >> 1) & 1, abort_flag, peer_abort, 12)) break;
+                if (!wait_bar(&bars[M_T0 + s], (c >> 1) & 1, abort_flag, peer_abort, 13)) break;
+                if (!wait_bar(&bars[M_ZREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 14)) break;
+                // the U columns are free once the epilogue has converted chunk c-1's U;
+                // the W columns once chunk c-1's -W has been read out
+                if (c >= 1 && !wait_bar(&bars[M_UCONV], (c - 1) & 1, abort_flag, peer_abort, 15)) break;
+                if (c >= 1 && !wait_bar(&bars[M_WFREE], (c - 1) & 1, abort_flag, peer_abort, 16)) break;
+                GDR2_TRACE_AT(c, 1);
                 tc_fence_after();
-                // [A^T | P^T] = Km [Em; Qm]^T   (M = 64 rows s, N = 128, lanes 0-15)
+                // W rows r (M = 64): key channels of block kb -> lanes 16 kb .. 16 kb + 15
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tb + kTmX, a, b, i_ap, kk > 0);
-                }
-                tc_commit(&bars[B_AP]);
-                GDR2_TRACE_AT(cp, 2);
-                if (!wait_bar(&bars[B_T], cp & 1, abort_flag, 14)) break;
-                // P^T read out of the shared columns (implies Z is ready): the W
-                // accumulator below shares those TMEM columns (other lanes)
-                if (!wait_bar(&bars[B_PREADY0 + s], (cp >> 1) & 1, abort_flag, 15)) break;
-                // the single U region is free once the epilogue has read chunk cp-1's U
-                if (cp >= 1 && !wait_bar(&bars[B_UCONV], (cp - 1) & 1, abort_flag, 16)) break;
-                tc_fence_after();
-                // W = T Em (M = 64 rows r, N = 128, lanes 16-31); U0^T = Z^T T^T (M = 128)
+                for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t at = smem_desc_sw128(tt + kk * 32, 16, 1024);
+                        const uint64_t be = smem_desc_sw128(eq + kb * 16384 + kk * 2048, 16384, 1024);
+                        mma_ss(tb + kTmW + ((uint32_t)(16 * kb) << 16), at, be, i_w, kk > 0);
+                    }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t at = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
-                    const uint64_t be = smem_desc_sw128(eq + kk * 2048, 16384, 1024);
-                    mma_ss(tb + kTmX + (16u << 16), at, be, i_w, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bt = smem_desc_sw128(sbase + kTB + kk * 32, 16, 1024);
-                    const uint64_t az = smem_desc_sw128(sbase + (s ? kZB1 : kZB0) + kk * 2048, 8192, 1024);
+                    const uint64_t bt = smem_desc_sw128(tt + kk * 32, 16, 1024);
+                    const uint64_t az = smem_desc_sw128(zz + kk * 2048, 8192, 1024);
                     mma_ss(tb + kTmU, az, bt, i_u, kk > 0);
                 }
-                tc_commit(&bars[B_WDONE]);
-                GDR2_TRACE_AT(cp, 3);
-                tc_commit(&bars[B_VFREE0 + s]);
+                tc_commit(&bars[M_WDONE]);
+                tc_commit(&bars[M_VFREE0 + s]);
+                GDR2_TRACE_AT(c, 2);
             }
-            // drain every MMA this thread issued before TMEM is released
-            tc_commit(&bars[B_DRAIN]);
-            volatile int dummy = 0;
-            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-            mbar_wait(&bars[B_DRAIN], 0, g2, 22);
+            tc_commit(&bars[M_DRAIN]);
+            drain_wait(&bars[M_DRAIN], 0, 22);
         }
-    } else if (warp == 3) {
-        // ---------------- MMA issuer for the state chain -----------------------
+    } else if (warp == 2) {
+        // ------------- relay: the helper's q, k, b slot may be reloaded ---------
+        // (its factors have landed here; only chunks the helper reloads after)
+        if (lane == 0) {
+            const uint32_t h_slotfree = mapa_shared(smem_u32(&bars[H_SLOTFREE0]), peer);
+            for (int c = 0; c + 2 < nc; ++c) {
+                const int s = c & 1;
+                if (!wait_bar(&bars[M_F0 + s], (c >> 1) & 1, abort_flag, peer_abort, 3)) break;
+                mbar_remote_arrive(h_slotfree + 8 * s);
+                GDR2_TRACE_AT(c, 3);
+            }
+        }
+    } else {
+        // ------------- MMA issuer: the state chain -----------------------------
         if (lane == 0) {
             const uint32_t i_uo = idesc_bf16_f32(128, 128, false, false);
             const uint32_t i_os = idesc_bf16_f32(128, 192, false, true);
-            for (int cc = 0; cc < nc; ++cc) {
-                const int s = cc & 1;
-                const uint32_t eq = sbase + (s ? kEQ1 : kEQ0);
-                const uint32_t kbs = sbase + (s ? kKB1 : kKB0);
-                if (!wait_bar(&bars[B_WREADY0 + s], (cc >> 1) & 1, abort_flag, 17)) break;
-                if (!wait_bar(&bars[B_SREADY], cc & 1, abort_flag, 18)) break;
-                GDR2_TRACE_AT(cc, 7);
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                const uint32_t eq = sbase + mEQ(s);
+                const uint32_t kbs = sbase + mKB(s);
+                if (!wait_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
+                if (!wait_bar(&bars[M_SREADY], c & 1, abort_flag, peer_abort, 18)) break;
+                GDR2_TRACE_AT(c, 4);
                 tc_fence_after();
                 // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows)
 #pragma unroll
@@ -419,11 +452,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                     mma_ts(tb + kTmU, tb + kTmSB + kk * 8, b, i_uo, 1);
                 }
-                tc_commit(&bars[B_UDONE]);
-                GDR2_TRACE_AT(cc, 4);
-                if (!wait_bar(&bars[B_UCONV], cc & 1, abort_flag, 19)) break;
-                if (!wait_bar(&bars[B_PREADY0 + s], (cc >> 1) & 1, abort_flag, 25)) break;
-                GDR2_TRACE_AT(cc, 6);
+                tc_commit(&bars[M_UDONE]);
+                GDR2_TRACE_AT(c, 5);
+                if (!wait_bar(&bars[M_UCONV], c & 1, abort_flag, peer_abort, 19)) break;
+                if (!wait_bar(&bars[M_P0 + s], (c >> 1) & 1, abort_flag, peer_abort, 25)) break;
+                GDR2_TRACE_AT(c, 6);
                 tc_fence_after();
                 // [O^T | M^T] += U^T [P^T | Km]   (N = 192, B MN-major: P^T atom, two Km atoms)
 #pragma unroll
@@ -431,99 +464,396 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     const uint64_t b = smem_desc_sw128(kbs + kk * 2048, 8192, 1024);
                     mma_ts(tb + kTmO, tb + kTmUB + kk * 8, b, i_os, 1);
                 }
-                tc_commit(&bars[B_SDONE]);
-                GDR2_TRACE_AT(cc, 5);
-                tc_commit(&bars[B_SLOTFREE0 + s]);
+                tc_commit(&bars[M_SDONE]);
+                tc_commit(&bars[M_SLOTFREE0 + s]);
+                GDR2_TRACE_AT(c, 7);
             }
-            tc_commit(&bars[B_DRAIN2]);
-            volatile int dummy = 0;
-            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-            mbar_wait(&bars[B_DRAIN2], 0, g2, 23);
+            tc_commit(&bars[M_DRAIN2]);
+            drain_wait(&bars[M_DRAIN2], 0, 23);
         }
     }
     } else if (warp < 8) {
         setmaxnreg_inc152();
-        // ---------------- prep A: decay factors, Z, P^T ------------------------
-        // Element-wise layout: lane g owns key channels 4g..4g+3 (64-channel
-        // block kb = g / 16), warp rb owns rows 16rb..16rb+15. Loads are
-        // unconditional (rows clamped to the valid range) and rows past the
-        // chunk end are zeroed with selects, so many loads stay in flight.
+        // ------------- Z = w . v, in place over the v tile ---------------------
+        // Lane g owns value channels 4g..4g+3 (64-channel block g / 16), warp pw
+        // rows 16pw..16pw+15; loads are unconditional (rows clamped) and rows
+        // past the chunk end are zeroed with selects.
         const int pw = warp - 4, tp = tid - 128;
-        const int g = lane, rb = pw, kb = g >> 4;
+        const int g = lane, kb = g >> 4;
         const uint32_t cbyte = 8 * (g & 15);
-        constexpr float kLog2e = 1.4426950408889634f;
-        const float *la_s = reinterpret_cast<const float *>(smem + kLA);  // staged log_alpha [64][128]
-        int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
-        if (tp == 0) {
-            ++la_issued;
-            mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
-            tma_load_3d(smem + kLA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)t_begin);
-        }
         for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            unsigned char *e_tile = smem + (s ? kEQ1 : kEQ0) + kb * 16384;
-            unsigned char *q_tile = e_tile + 8192;
-            unsigned char *k_tile = smem + (s ? kKB1 : kKB0) + kKmOff + kb * 8192;
-
-            if (tp == 0) GDR2_TRACE_AT(c, 8);
-            // write-gate rows of this chunk, consumed in the Z step (L2-prefetched)
             uint2 wv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int r = 16 * rb + i;
+                const int r = 16 * pw + i;
                 const int rr = r < L ? r : L - 1;
                 wv[i] = *reinterpret_cast<const uint2 *>(prm.w + ((t0 + rr) * H + h) * kD + 4 * g);
             }
-            if (!group_and(kBarPrepA, wait_bar(&bars[B_LAFULL], c & 1, abort_flag, 3))) break;
-            float4 la[16];
+            if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5)))
+                break;
+            unsigned char *z_tile = smem + mZ(s) + kb * 8192;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int r = 16 * rb + i;
+                const int r = 16 * pw + i;
+                const uint32_t off = sw128_offset(r, cbyte);
+                const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
+                const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
+                const float2 w0 = bf2_to_f2(wv[i].x), w1 = bf2_to_f2(wv[i].y);
+                const bool ok = r < L;
+                uint2 oz;
+                oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
+                oz.y = ok ? pack_bf16x2(v1.x * w1.x, v1.y * w1.y) : 0u;
+                *reinterpret_cast<uint2 *>(z_tile + off) = oz;
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarZ, 128);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 8);
+                mbar_arrive(&bars[M_ZREADY0 + s]);
+            }
+        }
+    } else if (warp < 12) {
+        setmaxnreg_inc152();
+        // ------------- -W, K-major, over the Em half of the slot -------------
+        // Warp pw reads its lane quarter of the W columns: lane i < 16 holds row
+        // r = 16 pw + i for key channels 0-63, lane 16 + i the same row for 64-127.
+        const int pw = warp - 8, tp = tid - 256;
+        const int rrow = 16 * pw + (lane & 15), kb = lane >> 4;
+        const uint32_t h_tfree = mapa_shared(smem_u32(&bars[H_TFREE0]), peer);
+        for (int c = 0; c < nc; ++c) {
+            const int s = c & 1;
+            if (!group_and(kBarW, 128, wait_bar(&bars[M_WDONE], c & 1, abort_flag, peer_abort, 8))) break;
+            // the W and U0 MMAs have read T: the helper may send chunk c + 2's T
+            // (only chunks the helper still sends wait for this)
+            if (tp == 0 && c + 2 < nc) mbar_remote_arrive(h_tfree + 8 * s);
+            GDR2_TRACE_AT(c, 9);
+            tc_fence_after();
+            uint32_t v0[32], v1[32];
+            const uint32_t taddr = tb + kTmW + ((uint32_t)(32 * pw) << 16);
+            tmem_ld32(taddr, v0);
+            tmem_ld32(taddr + 32, v1);
+            tc_wait_ld();
+            tc_fence_before();
+            float x[64];
+#pragma unroll
+            for (int j2 = 0; j2 < 32; ++j2) {
+                x[j2] = -__uint_as_float(v0[j2]);
+                x[32 + j2] = -__uint_as_float(v1[j2]);
+            }
+            store_row_bf16_sw128(smem + mEQ(s) + kb * 16384, rrow, x);
+            fence_proxy_async_smem();
+            named_bar_sync(kBarW, 128);
+            if (tp == 0) {
+                GDR2_TRACE_AT(c, 10);
+                mbar_arrive(&bars[M_WFREE]);
+                mbar_arrive(&bars[M_WREADY0 + s]);
+            }
+        }
+    } else {
+        setmaxnreg_inc152();
+        // ------------- epilogue ---------------------------------------------
+        const int ew = warp - 12, te = tid - 384;
+        const int j = 32 * ew + lane;                       // value channel = TMEM lane
+        const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
+        float *vecF = reinterpret_cast<float *>(smem + kM_VECF);
+        const uint32_t zeros[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                    0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        bool ok = true;
+        // master = Diag(e^{g_31 of chunk 0}) S0  (transposed: row j over key channels); O = 0
+        ok = group_and(kBarEpi, 128, wait_bar(&bars[M_F0], 0, abort_flag, peer_abort, 9));
+        if (ok) {
+            vecF[j] = expf(reinterpret_cast<const float *>(smem + mVEC(0))[j]);
+            named_bar_sync(kBarEpi, 128);
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4) {
+                uint32_t m[32], sbf[16];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int ch = 32 * g4 + q;
+                    const float s0 = prm.init_state ? prm.init_state[state_base + (int64_t)ch * kD + j] : 0.f;
+                    m[q] = __float_as_uint(vecF[ch] * s0);
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    sbf[q] = pack_bf16x2(__uint_as_float(m[2 * q]), __uint_as_float(m[2 * q + 1]));
+                tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
+                tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
+            }
+            tmem_st32(tb + kTmO + lane_off, zeros);
+            tmem_st32(tb + kTmO + lane_off + 32, zeros);
+            tc_wait_st();
+            tc_fence_before();
+            named_bar_sync(kBarEpi, 128);
+            if (te == 0) mbar_arrive(&bars[M_SREADY]);
+        }
+        for (int c = 0; ok && c < nc; ++c) {
+            const int s = c & 1;
+            const int64_t t0 = t_begin + 64 * c;
+            const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
+            // this chunk's second half sum (read now: the slot is refilled once
+            // the chunk's last MMA is done; the asm below makes the load complete
+            // before this thread passes the U hand-off that precedes that MMA)
+            float t1c = reinterpret_cast<const float *>(smem + mVEC(s))[128 + j];
+            asm volatile("mov.b32 %0, %0;" : "+f"(t1c));
+            // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
+            if (!group_and(kBarEpi, 128, wait_bar(&bars[M_UDONE], c & 1, abort_flag, peer_abort, 10))) break;
+            if (te == 0) GDR2_TRACE_AT(c, 11);
+            tc_fence_after();
+            {
+                uint32_t v0[32], v1[32], ub[16];
+                tmem_ld32(tb + kTmU + lane_off, v0);
+                tmem_ld32(tb + kTmU + lane_off + 32, v1);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    ub[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
+                tmem_st16(tb + kTmUB + lane_off, ub);
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    ub[q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
+                tmem_st16(tb + kTmUB + lane_off + 16, ub);
+                tc_wait_st();
+            }
+            tc_fence_before();
+            named_bar_sync(kBarEpi, 128);
+            if (te == 0) {
+                GDR2_TRACE_AT(c, 12);
+                mbar_arrive(&bars[M_UCONV]);
+            }
+
+            if (!group_and(kBarEpi, 128, wait_bar(&bars[M_SDONE], c & 1, abort_flag, peer_abort, 11))) break;
+            if (te == 0) GDR2_TRACE_AT(c, 13);
+            tc_fence_after();
+            // O^T row j -> registers as bf16 pairs (rows r, r+1), then the O region
+            // is zeroed for the next chunk; o is stored after the state hand-off
+            uint32_t opk[32];
+            {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tb + kTmO + lane_off, v0);
+                tmem_ld32(tb + kTmO + lane_off + 32, v1);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    opk[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
+                    opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
+                }
+            }
+            const bool last = (c + 1 == nc);
+            if (!last) {
+                tmem_st32(tb + kTmO + lane_off, zeros);
+                tmem_st32(tb + kTmO + lane_off + 32, zeros);
+            }
+            // state scale: e^{g_C - g_31} and, unless last, e^{g'_31} of the next chunk
+            // (the group barrier also means everyone is done reading vecF)
+            if (!group_and(kBarEpi, 128,
+                           last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag,
+                                                  peer_abort, 26)))
+                break;
+            vecF[j] = expf(t1c + (last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j]));
+            named_bar_sync(kBarEpi, 128);
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t m0[32], m1[32];
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 f0 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 4 * q);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 32 + 4 * q);
+                    m0[4 * q + 0] = __float_as_uint(__uint_as_float(m0[4 * q + 0]) * f0.x);
+                    m0[4 * q + 1] = __float_as_uint(__uint_as_float(m0[4 * q + 1]) * f0.y);
+                    m0[4 * q + 2] = __float_as_uint(__uint_as_float(m0[4 * q + 2]) * f0.z);
+                    m0[4 * q + 3] = __float_as_uint(__uint_as_float(m0[4 * q + 3]) * f0.w);
+                    m1[4 * q + 0] = __float_as_uint(__uint_as_float(m1[4 * q + 0]) * f1.x);
+                    m1[4 * q + 1] = __float_as_uint(__uint_as_float(m1[4 * q + 1]) * f1.y);
+                    m1[4 * q + 2] = __float_as_uint(__uint_as_float(m1[4 * q + 2]) * f1.z);
+                    m1[4 * q + 3] = __float_as_uint(__uint_as_float(m1[4 * q + 3]) * f1.w);
+                }
+                if (!last) {
+                    uint32_t s0b[16], s1b[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
+                        s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
+                    }
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
+                    tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
+                } else if (prm.final_state) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
+                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
+                    }
+                }
+            }
+            tc_wait_st();
+            tc_fence_before();
+            named_bar_sync(kBarEpi, 128);
+            if (te == 0) GDR2_TRACE_AT(c, 14);
+            if (!last && te == 0) mbar_arrive(&bars[M_SREADY]);
+            {   // o rows of this chunk: adjacent lanes (channels j, j+1) trade halves so
+                // that the even lane stores rows 2q and the odd lane rows 2q+1 as
+                // 4-byte (j, j+1) pairs
+                const bool odd = (lane & 1) != 0;
+                __nv_bfloat16 *obase = prm.o + (t0 * H + h) * kD + (j & ~1);
+                const int64_t rstride = H * kD;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel j
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
+                    const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+                    const int r = 2 * q + (odd ? 1 : 0);
+                    if (r < L) *reinterpret_cast<uint32_t *>(obase + r * rstride) = pr;
+                }
+            }
+        }
+    }
+    } else {
+    // =========================================================================
+    //                              helper CTA
+    // =========================================================================
+    if (warp < 4) {
+    setmaxnreg_dec40();
+    if (warp == 0) {
+        // ------------- q, k, b tiles ---------------------------------------------
+        if (lane == 0) {
+            int issued0 = 0, issued1 = 0;  // loads issued into each slot
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                if (c >= 2 &&
+                    !wait_bar(&bars[H_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
+                    break;
+                const int z = (int)(t_begin + 64 * c);
+                unsigned char *eq = smem + hEQ(s), *kq = smem + hEQ(s) + kH_KmOff;
+                GDR2_TRACE_AT(c, 16);
+                mbar_arrive_expect_tx(&bars[H_FULL0 + s], 3 * 16384);
+                for (int blk = 0; blk < 2; ++blk) {
+                    tma_load_3d(eq + blk * 16384, &map_b, &bars[H_FULL0 + s], 64 * blk, (int)h, z);
+                    tma_load_3d(eq + blk * 16384 + 8192, &map_q, &bars[H_FULL0 + s], 64 * blk, (int)h, z);
+                    tma_load_3d(kq + blk * 8192, &map_k, &bars[H_FULL0 + s], 64 * blk, (int)h, z);
+                }
+                (s ? issued1 : issued0) = (c >> 1) + 1;
+            }
+            if (issued0 > 0) drain_wait(&bars[H_FULL0], (issued0 - 1) & 1, 20);
+            if (issued1 > 0) drain_wait(&bars[H_FULL1], (issued1 - 1) & 1, 20);
+        }
+    } else if (warp == 1) {
+        // ------------- MMA issuer: [A^T | P^T] = Km [Em; Qm]^T ---------------
+        if (lane == 0) {
+            const uint32_t i_ap = idesc_bf16_f32(64, 128, false, false);
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                const uint32_t eq = sbase + hEQ(s);
+                const uint32_t km = eq + kH_KmOff;
+                if (!wait_bar(&bars[H_FDONE], c & 1, abort_flag, peer_abort, 12)) break;
+                if (c >= 2 && !wait_bar(&bars[H_XFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 13))
+                    break;
+                tc_fence_after();
+                // M = 64 rows s (lanes 0-15 of each quarter), N = 128: Em rows, then Qm rows
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tb + 128 * s, a, b, i_ap, kk > 0);
+                }
+                tc_commit(&bars[H_AP0 + s]);
+                tc_commit(&bars[H_SLOTFREE0 + s]);
+                GDR2_TRACE_AT(c, 17);
+            }
+            tc_commit(&bars[H_DRAIN]);
+            drain_wait(&bars[H_DRAIN], 0, 22);
+        }
+    }
+    } else if (warp < 12) {
+        setmaxnreg_inc152();
+        // ------------- decay factors, P^T (256 threads) ----------------------
+        // Element-wise layout: lane g owns key channels 4g..4g+3 (64-channel
+        // block kb = g / 16), warp pw owns rows 8pw..8pw+7. Rows past the chunk
+        // end are zeroed with selects. Software-pipelined: iteration c computes
+        // chunk c's factors and then reads out chunk c-1's P^T, so that the
+        // [A^T | P^T] MMA of a chunk runs while the next chunk's factors are
+        // computed.
+        const int pw = warp - 4, tp = tid - 128;
+        const int g = lane, kb = g >> 4;
+        const uint32_t cbyte = 8 * (g & 15);
+        constexpr float kLog2e = 1.4426950408889634f;
+        const float *la_s = reinterpret_cast<const float *>(smem + kH_LA);  // staged log_alpha [64][128]
+        float *vecBS = reinterpret_cast<float *>(smem + kH_BSUM);          // [8][128]
+        const uint32_t m_f = mapa_shared(smem_u32(&bars[M_F0]), peer);
+        const uint32_t m_p = mapa_shared(smem_u32(&bars[M_P0]), peer);
+        int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
+        if (tp == 0) {
+            ++la_issued;
+            mbar_arrive_expect_tx(&bars[H_LAFULL], 32768);
+            tma_load_3d(smem + kH_LA, &map_la, &bars[H_LAFULL], 0, (int)h, (int)t_begin);
+        }
+        for (int c = 0; c <= nc; ++c) {
+            const int s = c & 1;
+            const int64_t t0 = t_begin + 64 * c;
+            const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
+            if (c < nc) {
+            unsigned char *e_tile = smem + hEQ(s) + kb * 16384;
+            unsigned char *q_tile = e_tile + 8192;
+            unsigned char *k_tile = smem + hEQ(s) + kH_KmOff + kb * 8192;
+
+            if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_LAFULL], c & 1, abort_flag, peer_abort, 3))) break;
+            if (tp == 0) GDR2_TRACE_AT(c, 18);
+            float4 la[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * pw + i;
                 const float4 x = *reinterpret_cast<const float4 *>(la_s + r * 128 + 4 * g);
                 la[i] = r < L ? x : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             float4 bs = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 bs.x += la[i].x; bs.y += la[i].y; bs.z += la[i].z; bs.w += la[i].w;
             }
-            *reinterpret_cast<float4 *>(vecBS + rb * 128 + 4 * g) = bs;
-            if (tp == 0) GDR2_TRACE_AT(c, 9);
+            *reinterpret_cast<float4 *>(vecBS + pw * 128 + 4 * g) = bs;
             // (this group barrier also publishes the block sums and frees the staging tile)
             fence_proxy_async_smem();
-            if (!group_and(kBarPrepA, wait_bar(&bars[B_FULL0 + s], (c >> 1) & 1, abort_flag, 4))) break;
+            if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_FULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 4)))
+                break;
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 10);
+                GDR2_TRACE_AT(c, 19);
                 if (c + 1 < nc) {  // stage the next chunk's log_alpha
                     ++la_issued;
-                    mbar_arrive_expect_tx(&bars[B_LAFULL], 32768);
-                    tma_load_3d(smem + kLA, &map_la, &bars[B_LAFULL], 0, (int)h, (int)(t0 + 64));
+                    mbar_arrive_expect_tx(&bars[H_LAFULL], 32768);
+                    tma_load_3d(smem + kH_LA, &map_la, &bars[H_LAFULL], 0, (int)h, (int)(t0 + 64));
                 }
             }
             // d_r = g_r - g_31 in log2 units: suffix sums for rows < 32, prefix
             // sums for rows >= 32; half sums T0 = g_31, T1 = g_63 - g_31.
             {
-                float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (rb == 0) run = *reinterpret_cast<const float4 *>(vecBS + 1 * 128 + 4 * g);
-                if (rb == 3) run = *reinterpret_cast<const float4 *>(vecBS + 2 * 128 + 4 * g);
-                if (rb == 1 || rb == 2) {
-                    const float4 o4 = *reinterpret_cast<const float4 *>(vecBS + (rb == 1 ? 0 : 3) * 128 + 4 * g);
-                    float *vt = (rb == 1 ? vecT0 : vecT1) + (c & 3) * 128 + 4 * g;
-                    *reinterpret_cast<float4 *>(vt) =
-                        make_float4(bs.x + o4.x, bs.y + o4.y, bs.z + o4.z, bs.w + o4.w);
-                }
-                if (rb < 2) {
+                float4 run = make_float4(0.f, 0.f, 0.f, 0.f), half = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                    for (int i = 15; i >= 0; --i) {
+                for (int b = 0; b < 8; ++b) {
+                    const float4 o4 = *reinterpret_cast<const float4 *>(vecBS + b * 128 + 4 * g);
+                    const bool in_run = pw < 4 ? (b > pw && b < 4) : (b >= 4 && b < pw);
+                    const bool in_half = pw < 4 ? b < 4 : b >= 4;
+                    if (in_run) { run.x += o4.x; run.y += o4.y; run.z += o4.z; run.w += o4.w; }
+                    if (in_half) { half.x += o4.x; half.y += o4.y; half.z += o4.z; half.w += o4.w; }
+                }
+                if (pw == 0 || pw == 4)
+                    *reinterpret_cast<float4 *>(smem + hVEC(s) + (pw == 0 ? 0 : 512) + 16 * g) = half;
+                if (pw < 4) {
+#pragma unroll
+                    for (int i = 7; i >= 0; --i) {
                         const float4 x = la[i];
                         la[i] = make_float4(-run.x * kLog2e, -run.y * kLog2e, -run.z * kLog2e, -run.w * kLog2e);
                         run.x += x.x; run.y += x.y; run.z += x.z; run.w += x.w;
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         run.x += la[i].x; run.y += la[i].y; run.z += la[i].z; run.w += la[i].w;
                         la[i] = make_float4(run.x * kLog2e, run.y * kLog2e, run.z * kLog2e, run.w * kLog2e);
                     }
@@ -531,8 +861,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             // factors, in place: b -> Em, q -> Qm, k -> Km
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * rb + i;
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * pw + i;
                 const uint32_t off = sw128_offset(r, cbyte);
                 const uint2 qr = *reinterpret_cast<const uint2 *>(q_tile + off);
                 const uint2 kr = *reinterpret_cast<const uint2 *>(k_tile + off);
@@ -557,85 +887,92 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 *reinterpret_cast<uint2 *>(e_tile + off) = oe;
             }
             fence_proxy_async_smem();
-            named_bar_sync(kBarPrepA, 128);
+            named_bar_sync(kBarPrepA, 256);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 11);
-                mbar_arrive(&bars[B_PREP]);
-                mbar_arrive(&bars[B_VEC0 + s]);
-            }
-
-            // Z = w . v in place (v tile from TMA, w loaded at the chunk start)
-            {
-                if (!group_and(kBarPrepA, wait_bar(&bars[B_VFULL0 + s], (c >> 1) & 1, abort_flag, 5))) break;
-                unsigned char *z_tile = smem + (s ? kZB1 : kZB0) + kb * 8192;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int r = 16 * rb + i;
-                    const uint32_t off = sw128_offset(r, cbyte);
-                    const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
-                    const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
-                    const float2 w0 = bf2_to_f2(wv[i].x), w1 = bf2_to_f2(wv[i].y);
-                    const bool ok = r < L;
-                    uint2 oz;
-                    oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
-                    oz.y = ok ? pack_bf16x2(v1.x * w1.x, v1.y * w1.y) : 0u;
-                    *reinterpret_cast<uint2 *>(z_tile + off) = oz;
+                GDR2_TRACE_AT(c, 20);
+                mbar_arrive(&bars[H_FDONE]);
+                // Em, Qm, Km and the half sums to the main CTA, whose slot s is free
+                // once its chunk c-2 is fully consumed
+                if (c < 2 || wait_bar(&bars[H_MFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 7)) {
+                    const uint32_t bar = m_f + 8 * s;
+                    mbar_remote_arrive_expect_tx(bar, kFBytes);
+                    bulk_copy_to_cluster(mapa_shared(sbase + mEQ(s), peer), sbase + hEQ(s), 32768, bar);
+                    bulk_copy_to_cluster(mapa_shared(sbase + mKB(s) + kKmOff, peer), sbase + hEQ(s) + kH_KmOff,
+                                         16384, bar);
+                    bulk_copy_to_cluster(mapa_shared(sbase + mVEC(s), peer), sbase + hVEC(s), 1024, bar);
+                    copy_count[s] += 1;
+                    GDR2_TRACE_AT(c, 23);
                 }
             }
-            fence_proxy_async_smem();
-            named_bar_sync(kBarPrepA, 128);
-            if (tp == 0) {
-                GDR2_TRACE_AT(c, 12);
-                mbar_arrive(&bars[B_ZREADY0 + s]);
-            }
+            }  // c < nc
+            if (c == 0) continue;
 
-            // P^T[s][r] = P[r][s] (kept for s <= r) from the M=64 accumulator: lane
-            // i < 16 of warp pw holds row s = 16 pw + i -> MN-major rows before Km
-            if (!group_and(kBarPrepA, wait_bar(&bars[B_AP], c & 1, abort_flag, 6))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 13);
+            // P^T[s][r] = P[r][s] (kept for r >= s) of chunk cp = c - 1 from the M=64
+            // accumulator: lane i < 16 of a warp in lane quarter q holds row
+            // s = 16 q + i; the two warpgroups take the two 32-column halves
+            const int cp = c - 1, sp = cp & 1;
+            if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_AP0 + sp], (cp >> 1) & 1, abort_flag, peer_abort, 6)))
+                break;
+            if (tp == 0) GDR2_TRACE_AT(cp, 21);
             tc_fence_after();
             {
-                const uint32_t taddr = tb + kTmX + 64 + ((uint32_t)(32 * pw) << 16);
-                uint32_t v0[32], v1[32];
-                tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
+                const int q4 = pw & 3, hf = pw >> 2;
+                const uint32_t taddr = tb + 128 * sp + 64 + 32 * hf + ((uint32_t)(32 * q4) << 16);
+                uint32_t v[32];
+                tmem_ld32(taddr, v);
                 tc_wait_ld();
                 if (lane < 16) {
-                    const int srow = 16 * pw + lane;
-                    float x[64];
+                    const int srow = 16 * q4 + lane;
+                    unsigned char *pt = smem + hPT(sp);
 #pragma unroll
-                    for (int j2 = 0; j2 < 32; ++j2) {
-                        x[j2] = j2 >= srow ? __uint_as_float(v0[j2]) : 0.f;
-                        x[32 + j2] = 32 + j2 >= srow ? __uint_as_float(v1[j2]) : 0.f;
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int r0 = 32 * hf + 8 * q + 2 * e;
+                            u[e] = pack_bf16x2(r0 >= srow ? __uint_as_float(v[8 * q + 2 * e]) : 0.f,
+                                               r0 + 1 >= srow ? __uint_as_float(v[8 * q + 2 * e + 1]) : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(pt + sw128_offset(srow, 64 * hf + 16 * q)) =
+                            make_uint4(u[0], u[1], u[2], u[3]);
                     }
-                    store_row_bf16_sw128(smem + (s ? kKB1 : kKB0), srow, x);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar_sync(kBarPrepA, 128);
+            named_bar_sync(kBarPrepA, 256);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 14);
-                mbar_arrive(&bars[B_PREADY0 + s]);
+                GDR2_TRACE_AT(cp, 22);
+                mbar_arrive(&bars[H_XFREE0 + sp]);
+                // (the main CTA's buffer is free: chunk cp's factor copy already
+                // waited for chunk cp-2 to be consumed; so is this buffer's last
+                // content, chunk cp-2's P^T)
+                if (!*abort_flag) {
+                    const uint32_t bar = m_p + 8 * sp;
+                    mbar_remote_arrive_expect_tx(bar, 8192);
+                    bulk_copy_to_cluster(mapa_shared(sbase + mKB(sp), peer), sbase + hPT(sp), 8192, bar);
+                    copy_count[2 + sp] += 1;
+                }
             }
         }
-        if (tp == 0 && la_issued > 0) {  // drain a staged log_alpha load still in flight
-            volatile int dummy = 0;
-            WaitGuard g2{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
-            mbar_wait(&bars[B_LAFULL], (la_issued - 1) & 1, g2, 24);
-        }
-    } else if (warp < 12) {
+        if (tp == 0 && la_issued > 0)  // drain a staged log_alpha load still in flight
+            drain_wait(&bars[H_LAFULL], (la_issued - 1) & 1, 24);
+    } else {
         setmaxnreg_inc152();
-        // ---------------- prep B: (I + A)^{-1}, -W ------------------------------
-        const int pw = warp - 8, tp = tid - 256;
+        // ------------- (I + A)^{-1} ----------------------------------------------
+        const int pw = warp - 12, tp = tid - 384;
+        float *sA = reinterpret_cast<float *>(smem + kH_SA);
+        float *sT = reinterpret_cast<float *>(smem + kH_ST);
+        const uint32_t m_t = mapa_shared(smem_u32(&bars[M_T0]), peer);
         for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
-            if (!group_and(kBarPrepB, wait_bar(&bars[B_AP], c & 1, abort_flag, 7))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 15);
+            if (!group_and(kBarPrepB, 128, wait_bar(&bars[H_AP0 + s], (c >> 1) & 1, abort_flag, peer_abort, 8)))
+                break;
+            if (tp == 0) GDR2_TRACE_AT(c, 24);
             tc_fence_after();
             {   // A^T rows from the M=64 accumulator (lane i < 16 of warp pw: row s = 16 pw + i):
                 // A^T[s][r] = A[r][s], kept for r > s
-                const uint32_t taddr = tb + kTmX + ((uint32_t)(32 * pw) << 16);
+                const uint32_t taddr = tb + 128 * s + ((uint32_t)(32 * pw) << 16);
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
                 tmem_ld32(taddr + 32, v1);
@@ -663,11 +1000,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             named_bar_sync(kBarPrepB, 128);
             if (tp == 0) {
                 GDR2_TRACE_AT(c, 25);
-                // lanes 0-15 of the shared columns may now take the next [A^T | P^T]
-                // (prep A has read its P^T: that precedes PREP of the next chunk).
-                // The W readout below still loads all 32 lanes of each quarter,
-                // but it only uses lanes 16-31, which that MMA does not write.
-                mbar_arrive(&bars[B_AFREE]);
+                mbar_arrive(&bars[H_XFREE0 + s]);
             }
 
             // T = (I + A)^{-1} by doubling on 16-row blocks (A held transposed,
@@ -745,6 +1078,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             named_bar_sync(kBarPrepB, 128);
             if (tp == 0) GDR2_TRACE_AT(c, 27);
+            // T into the bf16 buffer: its previous content (chunk c-2) has reached the
+            // main CTA, and the main CTA's T buffer is free, once chunk c-2's W and U0
+            // MMAs are done
+            if (!group_and(kBarPrepB, 128,
+                           c < 2 || wait_bar(&bars[H_TFREE0 + s], ((c >> 1) - 1) & 1, abort_flag,
+                                                   peer_abort, 10)))
+                break;
+            if (tp == 0) GDR2_TRACE_AT(c, 28);
             {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
                 const int r = tp >> 1, half = tp & 1;
                 const float *trow = sT + r * kLD + 32 * half;
@@ -757,211 +1098,42 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         ue[e] = pack_bf16x2(s0 <= r ? trow[8 * q + 2 * e] : 0.f,
                                             s0 + 1 <= r ? trow[8 * q + 2 * e + 1] : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(smem + kTB + sw128_offset(r, 64 * half + 16 * q)) =
+                    *reinterpret_cast<uint4 *>(smem + hT(s) + sw128_offset(r, 64 * half + 16 * q)) =
                         make_uint4(ue[0], ue[1], ue[2], ue[3]);
                 }
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrepB, 128);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 16);
-                mbar_arrive(&bars[B_T]);
-            }
-
-            // W^T (lanes = key channels) -> -W, K-major, into the Em half of the slot
-            if (!group_and(kBarPrepB, wait_bar(&bars[B_WDONE], c & 1, abort_flag, 8))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 17);
-            tc_fence_after();
-            {   // W rows from the M=64 accumulator (lane 16 + i of warp pw: row r = 16 pw + i)
-                // -> -W, K-major, over the Em half of the slot (two 64-channel blocks)
-                const uint32_t taddr = tb + kTmX + ((uint32_t)(32 * pw) << 16);
-                const int rrow = 16 * pw + (lane & 15);
-#pragma unroll 1
-                for (int hb = 0; hb < 2; ++hb) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(taddr + 64 * hb, v0);
-                    tmem_ld32(taddr + 64 * hb + 32, v1);
-                    tc_wait_ld();
-                    if (lane >= 16) {
-                        float x[64];
-#pragma unroll
-                        for (int j2 = 0; j2 < 32; ++j2) {
-                            x[j2] = -__uint_as_float(v0[j2]);
-                            x[32 + j2] = -__uint_as_float(v1[j2]);
-                        }
-                        store_row_bf16_sw128(smem + (s ? kEQ1 : kEQ0) + hb * 16384, rrow, x);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(kBarPrepB, 128);
-            if (tp == 0) {
-                GDR2_TRACE_AT(c, 18);
-                mbar_arrive(&bars[B_WREADY0 + s]);
-            }
-        }
-    } else {
-        setmaxnreg_inc152();
-        // ---------------- epilogue warpgroup -----------------------------------
-        const int ew = warp - 12, te = tid - 384;
-        const int j = 32 * ew + lane;                       // value channel = TMEM lane
-        const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
-        const uint32_t zeros[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
-                                    0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        bool ok = true;
-        // master = Diag(e^{g_31 of chunk 0}) S0  (transposed: row j over key channels); O = 0
-        ok = group_and(kBarEpi, wait_bar(&bars[B_VEC0], 0, abort_flag, 9));
-        if (ok) {
-            vecF[j] = expf(vecT0[j]);
-            named_bar_sync(kBarEpi, 128);
-#pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4) {
-                uint32_t m[32], sbf[16];
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int ch = 32 * g4 + q;
-                    const float s0 = prm.init_state ? prm.init_state[state_base + (int64_t)ch * kD + j] : 0.f;
-                    m[q] = __float_as_uint(vecF[ch] * s0);
-                }
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    sbf[q] = pack_bf16x2(__uint_as_float(m[2 * q]), __uint_as_float(m[2 * q + 1]));
-                tmem_st32(tb + kTmMaster + lane_off + 32 * g4, m);
-                tmem_st16(tb + kTmSB + lane_off + 16 * g4, sbf);
-            }
-            tmem_st32(tb + kTmO + lane_off, zeros);
-            tmem_st32(tb + kTmO + lane_off + 32, zeros);
-            tc_wait_st();
-            tc_fence_before();
-            named_bar_sync(kBarEpi, 128);
-            if (te == 0) mbar_arrive(&bars[B_SREADY]);
-        }
-        for (int c = 0; ok && c < nc; ++c) {
-            const int64_t t0 = t_begin + 64 * c;
-            const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
-            if (!group_and(kBarEpi, wait_bar(&bars[B_UDONE], c & 1, abort_flag, 10))) break;
-            if (te == 0) GDR2_TRACE_AT(c, 20);
-            tc_fence_after();
-            {
-                uint32_t v0[32], v1[32], ub[16];
-                tmem_ld32(tb + kTmU + lane_off, v0);
-                tmem_ld32(tb + kTmU + lane_off + 32, v1);
-                tc_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    ub[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
-                tmem_st16(tb + kTmUB + lane_off, ub);
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    ub[q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
-                tmem_st16(tb + kTmUB + lane_off + 16, ub);
-                tc_wait_st();
-            }
-            tc_fence_before();
-            named_bar_sync(kBarEpi, 128);
-            if (te == 0) {
-                GDR2_TRACE_AT(c, 21);
-                mbar_arrive(&bars[B_UCONV]);
-            }
-
-            if (!group_and(kBarEpi, wait_bar(&bars[B_SDONE], c & 1, abort_flag, 11))) break;
-            if (te == 0) GDR2_TRACE_AT(c, 22);
-            tc_fence_after();
-            // O^T row j -> registers as bf16 pairs (rows r, r+1), then the O region
-            // is zeroed for the next chunk; o is stored after the state hand-off
-            uint32_t opk[32];
-            {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tb + kTmO + lane_off, v0);
-                tmem_ld32(tb + kTmO + lane_off + 32, v1);
-                tc_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    opk[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
-                    opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
-                }
-            }
-            const bool last = (c + 1 == nc);
-            if (!last) {
-                tmem_st32(tb + kTmO + lane_off, zeros);
-                tmem_st32(tb + kTmO + lane_off + 32, zeros);
-            }
-            if (te == 0) GDR2_TRACE_AT(c, 23);
-            // state scale: e^{g_C - g_31} and, unless last, e^{g'_31} of the next chunk
-            // (the group barrier also means everyone is done reading vecF)
-            if (!group_and(kBarEpi, last || wait_bar(&bars[B_VEC0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1,
-                                                      abort_flag, 26)))
-                break;
-            vecF[j] = expf(vecT1[(c & 3) * 128 + j] + (last ? 0.f : vecT0[((c + 1) & 3) * 128 + j]));
-            named_bar_sync(kBarEpi, 128);
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t m0[32], m1[32];
-                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                tmem_ld32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
-                tc_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 f0 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 4 * q);
-                    const float4 f1 = *reinterpret_cast<const float4 *>(vecF + 64 * hh + 32 + 4 * q);
-                    m0[4 * q + 0] = __float_as_uint(__uint_as_float(m0[4 * q + 0]) * f0.x);
-                    m0[4 * q + 1] = __float_as_uint(__uint_as_float(m0[4 * q + 1]) * f0.y);
-                    m0[4 * q + 2] = __float_as_uint(__uint_as_float(m0[4 * q + 2]) * f0.z);
-                    m0[4 * q + 3] = __float_as_uint(__uint_as_float(m0[4 * q + 3]) * f0.w);
-                    m1[4 * q + 0] = __float_as_uint(__uint_as_float(m1[4 * q + 0]) * f1.x);
-                    m1[4 * q + 1] = __float_as_uint(__uint_as_float(m1[4 * q + 1]) * f1.y);
-                    m1[4 * q + 2] = __float_as_uint(__uint_as_float(m1[4 * q + 2]) * f1.z);
-                    m1[4 * q + 3] = __float_as_uint(__uint_as_float(m1[4 * q + 3]) * f1.w);
-                }
-                if (!last) {
-                    uint32_t s0b[16], s1b[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
-                        s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
-                    }
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
-                    tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
-                    tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
-                } else if (prm.final_state) {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
-                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
-                    }
-                }
-            }
-            tc_wait_st();
-            tc_fence_before();
-            named_bar_sync(kBarEpi, 128);
-            if (te == 0) GDR2_TRACE_AT(c, 24);
-            if (!last && te == 0) mbar_arrive(&bars[B_SREADY]);
-            {   // o rows of this chunk: adjacent lanes (channels j, j+1) trade halves so
-                // that the even lane stores rows 2q and the odd lane rows 2q+1 as
-                // 4-byte (j, j+1) pairs
-                const bool odd = (lane & 1) != 0;
-                __nv_bfloat16 *obase = prm.o + (t0 * H + h) * kD + (j & ~1);
-                const int64_t rstride = H * kD;
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel j
-                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                    // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
-                    const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
-                    const int r = 2 * q + (odd ? 1 : 0);
-                    if (r < L) *reinterpret_cast<uint32_t *>(obase + r * rstride) = pr;
-                }
+                const uint32_t bar = m_t + 8 * s;
+                mbar_remote_arrive_expect_tx(bar, 8192);
+                bulk_copy_to_cluster(mapa_shared(sbase + mT(s), peer), sbase + hT(s), 8192, bar);
+                copy_count[4 + s] += 1;
+                GDR2_TRACE_AT(c, 29);
             }
         }
     }
+    }
 
+    // ---- teardown -----------------------------------------------------------
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // every copy and remote arrive of either CTA has been issued
+    if (is_main && tid == 0) {
+        // After an abort, copies from the helper may still be landing here: wait
+        // (bounded) for the last one the helper issued into each buffer.
+        const uint32_t cnt = mapa_shared(sbase + kMISC + 8, peer);
+        for (int s = 0; s < 2; ++s) {
+            const uint32_t n_f = ld_cluster_u32(cnt + 4 * s), n_p = ld_cluster_u32(cnt + 8 + 4 * s);
+            const uint32_t n_t = ld_cluster_u32(cnt + 16 + 4 * s);
+            if (n_f > 0) drain_wait(&bars[M_F0 + s], (n_f - 1) & 1, 27);
+            if (n_p > 0) drain_wait(&bars[M_P0 + s], (n_p - 1) & 1, 27);
+            if (n_t > 0) drain_wait(&bars[M_T0 + s], (n_t - 1) & 1, 28);
+        }
+    }
+    cluster_sync_all();
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(tb, 512);
+    if (tid == 0) GDR2_SPAN_AT(1, globaltimer_ns());
+    if (warp == 2) tmem_dealloc(tb, is_main ? 512 : 256);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -1007,9 +1179,10 @@ bool chunk_tc_supported(const ChunkArgs &a)
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
     const int64_t tokens = a.B * a.T;
-    const int64_t grid = a.num_seqs * a.H;
-    if (grid == 0) return cudaSuccess;
-    if (tokens > 0x7fffffffLL || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int64_t units = a.num_seqs * a.H;  // two CTAs per (sequence, head), kPairs pairs per cluster
+    if (units == 0) return cudaSuccess;
+    const int64_t clusters = (units + kPairs - 1) / kPairs;
+    if (tokens > 0x7fffffffLL || 2 * kPairs * clusters > 0x7fffffffLL) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mb, mv, mla, mw;
     const int64_t tk = tokens > 0 ? tokens : 1;
     const void *dummy = a.q ? a.q : (const void *)a.o;
@@ -1030,11 +1203,23 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.final_state = a.final_state;
     p.T = a.T;
     p.H = a.H;
+    p.units = units;
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<<<(unsigned)grid, kThreadsTC, kSmemBytes, stream>>>(mq, mk, mb, mv, mla, mw, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * kPairs * clusters), 1, 1);
+    cfg.blockDim = dim3(kThreadsTC, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2 * kPairs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk_tc_kernel, mq, mk, mb, mv, mla, mw, p);
 }
 
 namespace {

@@ -98,6 +98,8 @@ __host__ __device__ constexpr uint32_t mZ(int s) { return s ? 131072 : 114688; }
 __host__ __device__ constexpr uint32_t mT(int s) { return s ? 155648 : 147456; }     // T bf16, 64 rows x 128 B
 __host__ __device__ constexpr uint32_t mVEC(int s) { return s ? 164864 : 163840; }   // half sums [T0 | T1], fp32 128 + 128
 constexpr uint32_t kM_VECF = 165888;               // state scale factors, fp32 128
+constexpr uint32_t kM_OST = 166400;                // o staging: 64 rows of 256 B at a 320 B pitch
+constexpr uint32_t kOPitch = 320;                  // (row r+1 sits 16 banks after row r)
 // ---- helper CTA shared memory ----------------------------------------------
 __host__ __device__ constexpr uint32_t hEQ(int s) { return s ? 49152 : 0; }          // [b -> Em | q -> Qm] per key block, then k -> Km
 constexpr uint32_t kH_KmOff = 32768;
@@ -114,7 +116,7 @@ constexpr uint32_t kBAR = kH_BSUM + 8 * 128 * 4;   // same offset in both CTAs
 constexpr int kNumBars = 32;
 constexpr uint32_t kMISC = kBAR + kNumBars * 8;    // TMEM slot, abort flag, copy counters
 constexpr uint32_t kSmemBytes = kMISC + 64 + 1024; // + alignment slack
-static_assert(kM_VECF + 512 <= kBAR, "main shared-memory map overlaps the barriers");
+static_assert(kM_OST + 64 * kOPitch <= kBAR, "main shared-memory map overlaps the barriers");
 static_assert(kSmemBytes <= 232448, "shared memory above the per-CTA limit");
 
 constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
@@ -122,7 +124,8 @@ constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
 // barriers of the main CTA
 enum {
     M_F0 = 0, M_F1, M_P0, M_P1, M_T0, M_T1, M_VFULL0, M_VFULL1, M_VFREE0, M_VFREE1, M_ZREADY0, M_ZREADY1,
-    M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY, M_UDONE, M_UCONV, M_SDONE, M_SLOTFREE0,
+    M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY, M_UDONE, M_UCONV, M_SDONE, M_OFULL, M_OFREE,
+    M_SLOTFREE0,
     M_SLOTFREE1, M_DRAIN, M_DRAIN2, M_NUM
 };
 // barriers of the helper CTA
@@ -523,6 +526,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int pw = warp - 8, tp = tid - 256;
         const int rrow = 16 * pw + (lane & 15), kb = lane >> 4;
         const uint32_t h_tfree = mapa_shared(smem_u32(&bars[H_TFREE0]), peer);
+        // o of chunk cc from the staging tile: 16-byte pieces, 16 per row; rows
+        // past the sequence end are not written
+        auto store_o = [&](int cc) -> bool {
+            if (!group_and(kBarW, 128, wait_bar(&bars[M_OFULL], cc & 1, abort_flag, peer_abort, 30))) return false;
+            const int64_t t0 = t_begin + 64 * cc;
+            const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int idx = tp + 128 * i, r = idx >> 4, piece = idx & 15;
+                if (r < L) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(smem + kM_OST + r * kOPitch + 16 * piece);
+                    *reinterpret_cast<uint4 *>(prm.o + ((t0 + r) * H + h) * kD + 8 * piece) = v;
+                }
+            }
+            named_bar_sync(kBarW, 128);
+            if (tp == 0) mbar_arrive(&bars[M_OFREE]);
+            return true;
+        };
         for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
             if (!group_and(kBarW, 128, wait_bar(&bars[M_WDONE], c & 1, abort_flag, peer_abort, 8))) break;
@@ -551,6 +572,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_arrive(&bars[M_WFREE]);
                 mbar_arrive(&bars[M_WREADY0 + s]);
             }
+            // the previous chunk's o rows, staged by the epilogue
+            if (c >= 1 && !store_o(c - 1)) break;
+            if (c + 1 == nc) store_o(c);
         }
     } else {
         setmaxnreg_inc152();
@@ -697,12 +721,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             named_bar_sync(kBarEpi, 128);
             if (te == 0) GDR2_TRACE_AT(c, 14);
             if (!last && te == 0) mbar_arrive(&bars[M_SREADY]);
-            {   // o rows of this chunk: adjacent lanes (channels j, j+1) trade halves so
-                // that the even lane stores rows 2q and the odd lane rows 2q+1 as
-                // 4-byte (j, j+1) pairs
+            // o rows of this chunk into the staging tile, from which the -W group
+            // stores them to global memory; adjacent lanes (channels j, j+1) trade
+            // halves so that the even lane writes rows 2q and the odd lane rows
+            // 2q+1 as 4-byte (j, j+1) pairs
+            if (c >= 1 && !group_and(kBarEpi, 128, wait_bar(&bars[M_OFREE], (c - 1) & 1, abort_flag, peer_abort, 29)))
+                break;
+            {
                 const bool odd = (lane & 1) != 0;
-                __nv_bfloat16 *obase = prm.o + (t0 * H + h) * kD + (j & ~1);
-                const int64_t rstride = H * kD;
+                unsigned char *ost = smem + kM_OST + 2 * (j & ~1);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel j
@@ -710,9 +737,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
                     const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
                     const int r = 2 * q + (odd ? 1 : 0);
-                    if (r < L) *reinterpret_cast<uint32_t *>(obase + r * rstride) = pr;
+                    *reinterpret_cast<uint32_t *>(ost + r * kOPitch) = pr;
                 }
             }
+            named_bar_sync(kBarEpi, 128);
+            if (te == 0) mbar_arrive(&bars[M_OFULL]);
         }
     }
     } else {
@@ -770,6 +799,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tc_commit(&bars[H_DRAIN]);
             drain_wait(&bars[H_DRAIN], 0, 22);
         }
+    } else if (warp == 2) {
+        // ------------- factor sender: Em, Qm, Km, half sums -> main CTA ------
+        // (the main CTA's slot s is free once its chunk c-2 is fully consumed)
+        if (lane == 0) {
+            // (one CTA's window of the cluster's shared space is contiguous)
+            const uint32_t rbase = mapa_shared(sbase, peer);
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                if (!wait_bar(&bars[H_FDONE], c & 1, abort_flag, peer_abort, 14)) break;
+                if (c >= 2 && !wait_bar(&bars[H_MFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 15))
+                    break;
+                const uint32_t bar = rbase + kBAR + 8 * (M_F0 + s);
+                mbar_remote_arrive_expect_tx(bar, kFBytes);
+                bulk_copy_to_cluster(rbase + mEQ(s), sbase + hEQ(s), 32768, bar);
+                bulk_copy_to_cluster(rbase + mKB(s) + kKmOff, sbase + hEQ(s) + kH_KmOff, 16384, bar);
+                bulk_copy_to_cluster(rbase + mVEC(s), sbase + hVEC(s), 1024, bar);
+                copy_count[s] += 1;
+                GDR2_TRACE_AT(c, 23);
+            }
+        }
     }
     } else if (warp < 12) {
         setmaxnreg_inc152();
@@ -786,7 +835,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         constexpr float kLog2e = 1.4426950408889634f;
         const float *la_s = reinterpret_cast<const float *>(smem + kH_LA);  // staged log_alpha [64][128]
         float *vecBS = reinterpret_cast<float *>(smem + kH_BSUM);          // [8][128]
-        const uint32_t m_f = mapa_shared(smem_u32(&bars[M_F0]), peer);
         const uint32_t m_p = mapa_shared(smem_u32(&bars[M_P0]), peer);
         int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
         if (tp == 0) {
@@ -890,19 +938,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             named_bar_sync(kBarPrepA, 256);
             if (tp == 0) {
                 GDR2_TRACE_AT(c, 20);
-                mbar_arrive(&bars[H_FDONE]);
-                // Em, Qm, Km and the half sums to the main CTA, whose slot s is free
-                // once its chunk c-2 is fully consumed
-                if (c < 2 || wait_bar(&bars[H_MFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 7)) {
-                    const uint32_t bar = m_f + 8 * s;
-                    mbar_remote_arrive_expect_tx(bar, kFBytes);
-                    bulk_copy_to_cluster(mapa_shared(sbase + mEQ(s), peer), sbase + hEQ(s), 32768, bar);
-                    bulk_copy_to_cluster(mapa_shared(sbase + mKB(s) + kKmOff, peer), sbase + hEQ(s) + kH_KmOff,
-                                         16384, bar);
-                    bulk_copy_to_cluster(mapa_shared(sbase + mVEC(s), peer), sbase + hVEC(s), 1024, bar);
-                    copy_count[s] += 1;
-                    GDR2_TRACE_AT(c, 23);
-                }
+                mbar_arrive(&bars[H_FDONE]);  // to the MMA issuer and the factor sender
             }
             }  // c < nc
             if (c == 0) continue;
@@ -912,6 +948,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             // s = 16 q + i; the two warpgroups take the two 32-column halves
             const int cp = c - 1, sp = cp & 1;
             if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_AP0 + sp], (cp >> 1) & 1, abort_flag, peer_abort, 6)))
+                break;
+            // the P^T buffers here and in the main CTA hold chunk cp-2 until the main
+            // CTA has consumed it
+            if (!group_and(kBarPrepA, 256,
+                           cp < 2 || wait_bar(&bars[H_MFREE0 + sp], ((cp >> 1) - 1) & 1, abort_flag, peer_abort, 7)))
                 break;
             if (tp == 0) GDR2_TRACE_AT(cp, 21);
             tc_fence_after();
@@ -944,9 +985,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (tp == 0) {
                 GDR2_TRACE_AT(cp, 22);
                 mbar_arrive(&bars[H_XFREE0 + sp]);
-                // (the main CTA's buffer is free: chunk cp's factor copy already
-                // waited for chunk cp-2 to be consumed; so is this buffer's last
-                // content, chunk cp-2's P^T)
                 if (!*abort_flag) {
                     const uint32_t bar = m_p + 8 * sp;
                     mbar_remote_arrive_expect_tx(bar, 8192);

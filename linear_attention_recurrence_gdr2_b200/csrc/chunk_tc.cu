@@ -60,15 +60,16 @@ namespace gdr2 {
 
 __device__ int g_chunk_tc_error;
 
-// Optional per-phase SM-clock timestamps for the first CTAs (compiled in only
-// with -DGDR2_TRACE; the tracing driver points g_chunk_tc_trace at a buffer
-// of [4 CTAs][1024 chunks][32 events] uint64).
+// Optional per-phase SM-clock timestamps for CTAs 0-3 and 20-23 (compiled in
+// only with -DGDR2_TRACE; the tracing driver points g_chunk_tc_trace at a
+// buffer of [8 CTAs][1024 chunks][32 events] uint64).
 #ifdef GDR2_TRACE
 __device__ unsigned long long *g_chunk_tc_trace;
-#define GDR2_TRACE_AT(chunk, ev)                                                           \
-    do {                                                                                   \
-        if (blockIdx.x < 4 && g_chunk_tc_trace && (chunk) < 1024)                          \
-            g_chunk_tc_trace[((size_t)blockIdx.x * 1024 + (chunk)) * 32 + (ev)] = clock64(); \
+#define GDR2_TRACE_AT(chunk, ev)                                                                \
+    do {                                                                                        \
+        const unsigned ts_ = blockIdx.x < 4 ? blockIdx.x : blockIdx.x - 16;                     \
+        if (ts_ < 8 && g_chunk_tc_trace && (chunk) < 1024)                                      \
+            g_chunk_tc_trace[((size_t)ts_ * 1024 + (chunk)) * 32 + (ev)] = clock64();           \
     } while (0)
 // [CTA][start ns, end ns, SM id] for every CTA (buffer sized by the driver)
 __device__ unsigned long long *g_chunk_tc_span;
@@ -100,6 +101,7 @@ __host__ __device__ constexpr uint32_t mVEC(int s) { return s ? 164864 : 163840;
 constexpr uint32_t kM_VECF = 165888;               // state scale factors, fp32 128
 constexpr uint32_t kM_OST = 166400;                // o staging: 64 rows of 256 B at a 320 B pitch
 constexpr uint32_t kOPitch = 320;                  // (row r+1 sits 16 banks after row r)
+constexpr uint32_t kM_WT = 187392;                 // w tile (same layout as a v tile), 16 KB
 // ---- helper CTA shared memory ----------------------------------------------
 __host__ __device__ constexpr uint32_t hEQ(int s) { return s ? 49152 : 0; }          // [b -> Em | q -> Qm] per key block, then k -> Km
 constexpr uint32_t kH_KmOff = 32768;
@@ -116,7 +118,8 @@ constexpr uint32_t kBAR = kH_BSUM + 8 * 128 * 4;   // same offset in both CTAs
 constexpr int kNumBars = 32;
 constexpr uint32_t kMISC = kBAR + kNumBars * 8;    // TMEM slot, abort flag, copy counters
 constexpr uint32_t kSmemBytes = kMISC + 64 + 1024; // + alignment slack
-static_assert(kM_OST + 64 * kOPitch <= kBAR, "main shared-memory map overlaps the barriers");
+static_assert(kM_OST + 64 * kOPitch <= kM_WT && kM_WT + 16384 <= kBAR,
+              "main shared-memory map overlaps the barriers");
 static_assert(kSmemBytes <= 232448, "shared memory above the per-CTA limit");
 
 constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
@@ -125,6 +128,7 @@ constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
 enum {
     M_F0 = 0, M_F1, M_P0, M_P1, M_T0, M_T1, M_VFULL0, M_VFULL1, M_VFREE0, M_VFREE1, M_ZREADY0, M_ZREADY1,
     M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY, M_UDONE, M_UCONV, M_SDONE, M_OFULL, M_OFREE,
+    M_WTFULL, M_WTFREE,
     M_SLOTFREE0,
     M_SLOTFREE1, M_DRAIN, M_DRAIN2, M_NUM
 };
@@ -172,6 +176,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     if (!ok) st_cluster_u32(peer_abort, 1u);
     return ok;
 }
+
+// Descriptor of the operand `bytes` further on in the same tile (the start
+// address field is the low 14 bits in 16-byte units and shared addresses stay
+// below 256 KB, so this adds without a carry out of the field).
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // Bounded wait used only while winding down (never raises the abort flag).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int site) {
@@ -358,11 +367,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     if (warp < 4) {
     setmaxnreg_dec40();
     if (warp == 0) {
-        // ------------- v tiles, L2 prefetch of w, slot-free relay -------------
+        // ------------- v and w tiles, slot-free relay ------------------------
         if (lane == 0) {
             const uint32_t h_mfree = mapa_shared(smem_u32(&bars[H_MFREE0]), peer);
-            tma_prefetch_3d(&map_w, 0, (int)h, (int)t_begin);
             int vissued0 = 0, vissued1 = 0;  // loads issued into each slot
+            int wissued = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
                 if (c >= 2 && !wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
@@ -373,7 +382,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 for (int blk = 0; blk < 2; ++blk)
                     tma_load_3d(smem + mZ(s) + blk * 8192, &map_v, &bars[M_VFULL0 + s], 64 * blk, (int)h, z);
                 (s ? vissued1 : vissued0) = (c >> 1) + 1;
-                if (c + 1 < nc) tma_prefetch_3d(&map_w, 0, (int)h, z + 64);
+                // the single w buffer: free once Z of chunk c-1 is done
+                if (c >= 1 && !wait_bar(&bars[M_WTFREE], (c - 1) & 1, abort_flag, peer_abort, 4)) break;
+                mbar_arrive_expect_tx(&bars[M_WTFULL], 16384);
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_load_3d(smem + kM_WT + blk * 8192, &map_w, &bars[M_WTFULL], 64 * blk, (int)h, z);
+                ++wissued;
                 // slot s of chunk c - 2 fully consumed (its last MMA is done):
                 // the helper may copy chunk c into it
                 if (c >= 2) {
@@ -384,15 +398,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             if (vissued0 > 0) drain_wait(&bars[M_VFULL0], (vissued0 - 1) & 1, 20);
             if (vissued1 > 0) drain_wait(&bars[M_VFULL1], (vissued1 - 1) & 1, 20);
+            if (wissued > 0) drain_wait(&bars[M_WTFULL], (wissued - 1) & 1, 21);
         }
     } else if (warp == 1) {
         // ------------- MMA issuer: W = T Em, U0^T = Z^T T^T --------------------
         if (lane == 0) {
-            const uint32_t i_w = idesc_bf16_f32(64, 64, false, true);
+            const uint32_t i_w = idesc_bf16_f32(64, 64, false, true, true);  // -(T Em)
             const uint32_t i_u = idesc_bf16_f32(128, 64, true, false);
+            const uint64_t d_t = smem_desc_sw128(sbase + mT(0), 16, 1024);
+            const uint64_t d_em = smem_desc_sw128(sbase + mEQ(0), 16384, 1024);
+            const uint64_t d_z = smem_desc_sw128(sbase + mZ(0), 8192, 1024);
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                const uint32_t eq = sbase + mEQ(s), tt = sbase + mT(s), zz = sbase + mZ(s);
+                const uint64_t dt = desc_at(d_t, mT(s) - mT(0)), dem = desc_at(d_em, mEQ(s) - mEQ(0));
+                const uint64_t dz = desc_at(d_z, mZ(s) - mZ(0));
                 if (!wait_bar(&bars[M_F0 + s], (c >> 1) & 1, abort_flag, peer_abort, 12)) break;
                 if (!wait_bar(&bars[M_T0 + s], (c >> 1) & 1, abort_flag, peer_abort, 13)) break;
                 if (!wait_bar(&bars[M_ZREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 14)) break;
@@ -402,21 +421,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 if (c >= 1 && !wait_bar(&bars[M_WFREE], (c - 1) & 1, abort_flag, peer_abort, 16)) break;
                 GDR2_TRACE_AT(c, 1);
                 tc_fence_after();
-                // W rows r (M = 64): key channels of block kb -> lanes 16 kb .. 16 kb + 15
+                // -W rows r (M = 64, A negated): key channels of block kb -> lanes 16 kb .. 16 kb + 15
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t at = smem_desc_sw128(tt + kk * 32, 16, 1024);
-                        const uint64_t be = smem_desc_sw128(eq + kb * 16384 + kk * 2048, 16384, 1024);
-                        mma_ss(tb + kTmW + ((uint32_t)(16 * kb) << 16), at, be, i_w, kk > 0);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tb + kTmW + ((uint32_t)(16 * kb) << 16), desc_at(dt, kk * 32),
+                               desc_at(dem, kb * 16384 + kk * 2048), i_w, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bt = smem_desc_sw128(tt + kk * 32, 16, 1024);
-                    const uint64_t az = smem_desc_sw128(zz + kk * 2048, 8192, 1024);
-                    mma_ss(tb + kTmU, az, bt, i_u, kk > 0);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tb + kTmU, desc_at(dz, kk * 2048), desc_at(dt, kk * 32), i_u, kk > 0);
                 tc_commit(&bars[M_WDONE]);
                 tc_commit(&bars[M_VFREE0 + s]);
                 GDR2_TRACE_AT(c, 2);
@@ -441,20 +455,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         if (lane == 0) {
             const uint32_t i_uo = idesc_bf16_f32(128, 128, false, false);
             const uint32_t i_os = idesc_bf16_f32(128, 192, false, true);
+            const uint64_t d_wq = smem_desc_sw128(sbase + mEQ(0), 16, 1024);
+            const uint64_t d_pk = smem_desc_sw128(sbase + mKB(0), 8192, 1024);
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                const uint32_t eq = sbase + mEQ(s);
-                const uint32_t kbs = sbase + mKB(s);
+                const uint64_t dwq = desc_at(d_wq, mEQ(s) - mEQ(0)), dpk = desc_at(d_pk, mKB(s) - mKB(0));
                 if (!wait_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
                 if (!wait_bar(&bars[M_SREADY], c & 1, abort_flag, peer_abort, 18)) break;
                 GDR2_TRACE_AT(c, 4);
                 tc_fence_after();
                 // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, b, i_uo, 1);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, desc_at(dwq, (kk >> 2) * 16384 + (kk & 3) * 32), i_uo, 1);
                 tc_commit(&bars[M_UDONE]);
                 GDR2_TRACE_AT(c, 5);
                 if (!wait_bar(&bars[M_UCONV], c & 1, abort_flag, peer_abort, 19)) break;
@@ -463,10 +476,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 tc_fence_after();
                 // [O^T | M^T] += U^T [P^T | Km]   (N = 192, B MN-major: P^T atom, two Km atoms)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t b = smem_desc_sw128(kbs + kk * 2048, 8192, 1024);
-                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, b, i_os, 1);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tb + kTmO, tb + kTmUB + kk * 8, desc_at(dpk, kk * 2048), i_os, 1);
                 tc_commit(&bars[M_SDONE]);
                 tc_commit(&bars[M_SLOTFREE0 + s]);
                 GDR2_TRACE_AT(c, 7);
@@ -479,8 +490,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         setmaxnreg_inc152();
         // ------------- Z = w . v, in place over the v tile ---------------------
         // Lane g owns value channels 4g..4g+3 (64-channel block g / 16), warp pw
-        // rows 16pw..16pw+15; loads are unconditional (rows clamped) and rows
-        // past the chunk end are zeroed with selects.
+        // rows 16pw..16pw+15; rows past the chunk end are zeroed.
         const int pw = warp - 4, tp = tid - 128;
         const int g = lane, kb = g >> 4;
         const uint32_t cbyte = 8 * (g & 15);
@@ -488,23 +498,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            uint2 wv[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * pw + i;
-                const int rr = r < L ? r : L - 1;
-                wv[i] = *reinterpret_cast<const uint2 *>(prm.w + ((t0 + rr) * H + h) * kD + 4 * g);
-            }
-            if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5)))
+            if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5) &&
+                                           wait_bar(&bars[M_WTFULL], c & 1, abort_flag, peer_abort, 6)))
                 break;
             unsigned char *z_tile = smem + mZ(s) + kb * 8192;
-#pragma unroll
+            const unsigned char *w_tile = smem + kM_WT + kb * 8192;
+#pragma unroll 4
             for (int i = 0; i < 16; ++i) {
                 const int r = 16 * pw + i;
                 const uint32_t off = sw128_offset(r, cbyte);
                 const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
+                const uint2 wr = *reinterpret_cast<const uint2 *>(w_tile + off);
                 const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
-                const float2 w0 = bf2_to_f2(wv[i].x), w1 = bf2_to_f2(wv[i].y);
+                const float2 w0 = bf2_to_f2(wr.x), w1 = bf2_to_f2(wr.y);
                 const bool ok = r < L;
                 uint2 oz;
                 oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
@@ -516,12 +522,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (tp == 0) {
                 GDR2_TRACE_AT(c, 8);
                 mbar_arrive(&bars[M_ZREADY0 + s]);
+                mbar_arrive(&bars[M_WTFREE]);
             }
         }
     } else if (warp < 12) {
         setmaxnreg_inc152();
         // ------------- -W, K-major, over the Em half of the slot -------------
-        // Warp pw reads its lane quarter of the W columns: lane i < 16 holds row
+        // Warp pw reads its lane quarter of the -W columns: lane i < 16 holds row
         // r = 16 pw + i for key channels 0-63, lane 16 + i the same row for 64-127.
         const int pw = warp - 8, tp = tid - 256;
         const int rrow = 16 * pw + (lane & 15), kb = lane >> 4;
@@ -544,8 +551,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (tp == 0) mbar_arrive(&bars[M_OFREE]);
             return true;
         };
-        for (int c = 0; c < nc; ++c) {
+        for (int c = 0; c <= nc; ++c) {
             const int s = c & 1;
+            if (c < nc) {
             if (!group_and(kBarW, 128, wait_bar(&bars[M_WDONE], c & 1, abort_flag, peer_abort, 8))) break;
             // the W and U0 MMAs have read T: the helper may send chunk c + 2's T
             // (only chunks the helper still sends wait for this)
@@ -561,8 +569,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             float x[64];
 #pragma unroll
             for (int j2 = 0; j2 < 32; ++j2) {
-                x[j2] = -__uint_as_float(v0[j2]);
-                x[32 + j2] = -__uint_as_float(v1[j2]);
+                x[j2] = __uint_as_float(v0[j2]);
+                x[32 + j2] = __uint_as_float(v1[j2]);
             }
             store_row_bf16_sw128(smem + mEQ(s) + kb * 16384, rrow, x);
             fence_proxy_async_smem();
@@ -572,9 +580,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_arrive(&bars[M_WFREE]);
                 mbar_arrive(&bars[M_WREADY0 + s]);
             }
+            }  // c < nc
             // the previous chunk's o rows, staged by the epilogue
             if (c >= 1 && !store_o(c - 1)) break;
-            if (c + 1 == nc) store_o(c);
         }
     } else {
         setmaxnreg_inc152();
@@ -777,21 +785,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         // ------------- MMA issuer: [A^T | P^T] = Km [Em; Qm]^T ---------------
         if (lane == 0) {
             const uint32_t i_ap = idesc_bf16_f32(64, 128, false, false);
+            const uint64_t d_km = smem_desc_sw128(sbase + hEQ(0) + kH_KmOff, 16, 1024);
+            const uint64_t d_eq = smem_desc_sw128(sbase + hEQ(0), 16, 1024);
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                const uint32_t eq = sbase + hEQ(s);
-                const uint32_t km = eq + kH_KmOff;
+                const uint64_t dkm = desc_at(d_km, hEQ(s) - hEQ(0)), deq = desc_at(d_eq, hEQ(s) - hEQ(0));
                 if (!wait_bar(&bars[H_FDONE], c & 1, abort_flag, peer_abort, 12)) break;
                 if (c >= 2 && !wait_bar(&bars[H_XFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 13))
                     break;
                 tc_fence_after();
                 // M = 64 rows s (lanes 0-15 of each quarter), N = 128: Em rows, then Qm rows
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = smem_desc_sw128(km + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(eq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tb + 128 * s, a, b, i_ap, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tb + 128 * s, desc_at(dkm, (kk >> 2) * 8192 + (kk & 3) * 32),
+                           desc_at(deq, (kk >> 2) * 16384 + (kk & 3) * 32), i_ap, kk > 0);
                 tc_commit(&bars[H_AP0 + s]);
                 tc_commit(&bars[H_SLOTFREE0 + s]);
                 GDR2_TRACE_AT(c, 17);
@@ -1229,7 +1236,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
               make_map(&mb, a.b ? a.b : dummy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tk, a.H, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&mv, a.v ? a.v : dummy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tk, a.H, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&mla, a.log_alpha ? (const void *)a.log_alpha : dummy, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tk, a.H, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              make_map(&mw, a.w ? a.w : dummy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tk, a.H, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+              make_map(&mw, a.w ? a.w : dummy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tk, a.H, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     TcParams p;
     p.la = a.log_alpha;

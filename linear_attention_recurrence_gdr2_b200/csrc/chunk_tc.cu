@@ -127,7 +127,8 @@ constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
 // barriers of the main CTA
 enum {
     M_F0 = 0, M_F1, M_P0, M_P1, M_T0, M_T1, M_VFULL0, M_VFULL1, M_VFREE0, M_VFREE1, M_ZREADY0, M_ZREADY1,
-    M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY, M_UDONE, M_UCONV, M_SDONE, M_OFULL, M_OFREE,
+    M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY_LO, M_SREADY_HI, M_UDONE, M_UCONV, M_SDONE,
+    M_OFULL, M_OFREE,
     M_WTFULL, M_WTFREE,
     M_SLOTFREE0,
     M_SLOTFREE1, M_DRAIN, M_DRAIN2, M_NUM
@@ -171,7 +172,7 @@ struct TcParams {
 // flag, so that the whole cluster winds down.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                          uint32_t peer_abort, int site) {
-    WaitGuard g{globaltimer_ns() + kWaitNs, abort_flag, &g_chunk_tc_error};
+    WaitGuard g{kWaitNs, abort_flag, &g_chunk_tc_error};
     const bool ok = mbar_wait(bar, parity, g, site);
     if (!ok) st_cluster_u32(peer_abort, 1u);
     return ok;
@@ -182,10 +183,33 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
 // below 256 KB, so this adds without a carry out of the field).
 __device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
+// Bounded wait that polls without suspending, for the state-chain MMA issuer
+// (a suspended wait adds its wake-up time to every chunk).
+__device__ __forceinline__ bool spin_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         uint32_t peer_abort, int site) {
+    uint64_t deadline = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 255u) == 255u) {
+            if (*abort_flag) break;
+            const uint64_t now = globaltimer_ns();
+            if (deadline == 0) {
+                deadline = now + kWaitNs;
+            } else if (now > deadline) {
+                *abort_flag = 1;
+                atomicCAS(&g_chunk_tc_error, 0, 0x100 | site);
+                break;
+            }
+        }
+    }
+    st_cluster_u32(peer_abort, 1u);
+    return false;
+}
+
 // Bounded wait used only while winding down (never raises the abort flag).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int site) {
     volatile int dummy = 0;
-    WaitGuard g{globaltimer_ns() + kWaitNs, &dummy, &g_chunk_tc_error};
+    WaitGuard g{kWaitNs, &dummy, &g_chunk_tc_error};
     mbar_wait(bar, parity, g, site);
 }
 
@@ -202,11 +226,10 @@ __device__ __forceinline__ bool group_and(uint32_t id, uint32_t n, bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// An fp32 value as a tf32 MMA operand: the tensor core reads only the tf32
+// bits (sign, exponent, 10 mantissa bits), i.e. the value truncated toward
+// zero (relative error below 2^-10; T is consumed in bf16, 2^-9).
+__device__ __forceinline__ uint32_t to_tf32(float x) { return __float_as_uint(x); }
 // Warp-level D (16x8, fp32) += A (16x8, tf32) * B (8x8, tf32).
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -222,7 +245,7 @@ template <int K>
 __device__ __forceinline__ void tile_tf32(float (&d)[4], const float *x, int xsi, int xsk,
                                           const float *y, int ysk, int lane) {
     const int ar = lane >> 2, ac = lane & 3;
-#pragma unroll
+#pragma unroll 2
     for (int k0 = 0; k0 < K; k0 += 8) {
         uint32_t a[4], b[2];
         a[0] = to_tf32(x[ar * xsi + (k0 + ac) * xsk]);
@@ -460,18 +483,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
                 const uint64_t dwq = desc_at(d_wq, mEQ(s) - mEQ(0)), dpk = desc_at(d_pk, mKB(s) - mKB(0));
-                if (!wait_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
-                if (!wait_bar(&bars[M_SREADY], c & 1, abort_flag, peer_abort, 18)) break;
+                if (!spin_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
+                if (!spin_bar(&bars[M_SREADY_LO], c & 1, abort_flag, peer_abort, 18)) break;
                 GDR2_TRACE_AT(c, 4);
                 tc_fence_after();
-                // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows)
+                // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows); the
+                // state arrives in two halves of 64 key channels (K steps 0-3, 4-7)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, desc_at(dwq, (kk >> 2) * 16384 + (kk & 3) * 32), i_uo, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, desc_at(dwq, (kk & 3) * 32), i_uo, 1);
+                if (!spin_bar(&bars[M_SREADY_HI], c & 1, abort_flag, peer_abort, 24)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
+                    mma_ts(tb + kTmU, tb + kTmSB + kk * 8, desc_at(dwq, 16384 + (kk & 3) * 32), i_uo, 1);
                 tc_commit(&bars[M_UDONE]);
                 GDR2_TRACE_AT(c, 5);
-                if (!wait_bar(&bars[M_UCONV], c & 1, abort_flag, peer_abort, 19)) break;
-                if (!wait_bar(&bars[M_P0 + s], (c >> 1) & 1, abort_flag, peer_abort, 25)) break;
+                if (!spin_bar(&bars[M_UCONV], c & 1, abort_flag, peer_abort, 19)) break;
+                if (!spin_bar(&bars[M_P0 + s], (c >> 1) & 1, abort_flag, peer_abort, 25)) break;
                 GDR2_TRACE_AT(c, 6);
                 tc_fence_after();
                 // [O^T | M^T] += U^T [P^T | Km]   (N = 192, B MN-major: P^T atom, two Km atoms)
@@ -619,7 +648,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tc_wait_st();
             tc_fence_before();
             named_bar_sync(kBarEpi, 128);
-            if (te == 0) mbar_arrive(&bars[M_SREADY]);
+            if (te == 0) {
+                mbar_arrive(&bars[M_SREADY_LO]);
+                mbar_arrive(&bars[M_SREADY_HI]);
+            }
         }
         for (int c = 0; ok && c < nc; ++c) {
             const int s = c & 1;
@@ -630,6 +662,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             // before this thread passes the U hand-off that precedes that MMA)
             float t1c = reinterpret_cast<const float *>(smem + mVEC(s))[128 + j];
             asm volatile("mov.b32 %0, %0;" : "+f"(t1c));
+            const bool last = (c + 1 == nc);
+            // state scale for this chunk's hand-off, e^{g_C - g_31} and, unless last,
+            // e^{g'_31} of the next chunk (whose factors arrived long ago); the last
+            // readers of vecF finished before the previous chunk's final group barrier
+            if (!group_and(kBarEpi, 128,
+                           last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag, peer_abort, 26)))
+                break;
+            vecF[j] = expf(t1c + (last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j]));
             // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_UDONE], c & 1, abort_flag, peer_abort, 10))) break;
             if (te == 0) GDR2_TRACE_AT(c, 11);
@@ -673,19 +713,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
                 }
             }
-            const bool last = (c + 1 == nc);
             if (!last) {
                 tmem_st32(tb + kTmO + lane_off, zeros);
                 tmem_st32(tb + kTmO + lane_off + 32, zeros);
             }
-            // state scale: e^{g_C - g_31} and, unless last, e^{g'_31} of the next chunk
-            // (the group barrier also means everyone is done reading vecF)
-            if (!group_and(kBarEpi, 128,
-                           last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag,
-                                                  peer_abort, 26)))
-                break;
-            vecF[j] = expf(t1c + (last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j]));
-            named_bar_sync(kBarEpi, 128);
+            // the state, scaled, in two halves of 64 key channels: each half is
+            // handed to the chain as soon as its bf16 copy is in TMEM
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t m0[32], m1[32];
@@ -712,10 +745,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         s0b[q] = pack_bf16x2(__uint_as_float(m0[2 * q]), __uint_as_float(m0[2 * q + 1]));
                         s1b[q] = pack_bf16x2(__uint_as_float(m1[2 * q]), __uint_as_float(m1[2 * q + 1]));
                     }
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
                     tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
                     tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
+                    tc_wait_st();
+                    tc_fence_before();
+                    named_bar_sync(kBarEpi, 128);
+                    if (te == 0) mbar_arrive(&bars[hh ? M_SREADY_HI : M_SREADY_LO]);
                 } else if (prm.final_state) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) {
@@ -724,11 +761,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     }
                 }
             }
-            tc_wait_st();
-            tc_fence_before();
-            named_bar_sync(kBarEpi, 128);
             if (te == 0) GDR2_TRACE_AT(c, 14);
-            if (!last && te == 0) mbar_arrive(&bars[M_SREADY]);
             // o rows of this chunk into the staging tile, from which the -W group
             // stores them to global memory; adjacent lanes (channels j, j+1) trade
             // halves so that the even lane writes rows 2q and the odd lane rows
@@ -1016,28 +1049,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (tp == 0) GDR2_TRACE_AT(c, 24);
             tc_fence_after();
             {   // A^T rows from the M=64 accumulator (lane i < 16 of warp pw: row s = 16 pw + i):
-                // A^T[s][r] = A[r][s], kept for r > s
+                // A^T[s][r] = A[r][s] for r > s
                 const uint32_t taddr = tb + 128 * s + ((uint32_t)(32 * pw) << 16);
-                uint32_t v0[32], v1[32];
-                tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
-                tc_wait_ld();
-                if (lane < 16) {
-                    const int srow = 16 * pw + lane;
-                    float *row = sA + srow * kLD;
+                // (entries with r <= s are left as computed: the solve below reads
+                // only the strictly lower triangle of A)
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 a0, a1;
-                        a0.x = 4 * q + 0 > srow ? __uint_as_float(v0[4 * q + 0]) : 0.f;
-                        a0.y = 4 * q + 1 > srow ? __uint_as_float(v0[4 * q + 1]) : 0.f;
-                        a0.z = 4 * q + 2 > srow ? __uint_as_float(v0[4 * q + 2]) : 0.f;
-                        a0.w = 4 * q + 3 > srow ? __uint_as_float(v0[4 * q + 3]) : 0.f;
-                        a1.x = 32 + 4 * q + 0 > srow ? __uint_as_float(v1[4 * q + 0]) : 0.f;
-                        a1.y = 32 + 4 * q + 1 > srow ? __uint_as_float(v1[4 * q + 1]) : 0.f;
-                        a1.z = 32 + 4 * q + 2 > srow ? __uint_as_float(v1[4 * q + 2]) : 0.f;
-                        a1.w = 32 + 4 * q + 3 > srow ? __uint_as_float(v1[4 * q + 3]) : 0.f;
-                        *reinterpret_cast<float4 *>(row + 4 * q) = a0;
-                        *reinterpret_cast<float4 *>(row + 32 + 4 * q) = a1;
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + 32 * hf, v);
+                    tc_wait_ld();
+                    if (lane < 16) {
+                        float *row = sA + (16 * pw + lane) * kLD + 32 * hf;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<uint4 *>(row + 4 * q) =
+                                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
                 }
             }
@@ -1281,7 +1307,7 @@ __global__ void wait_selftest_kernel(uint64_t timeout_ns)
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        WaitGuard g{globaltimer_ns() + timeout_ns, &abort_flag, &g_chunk_tc_error};
+        WaitGuard g{timeout_ns, &abort_flag, &g_chunk_tc_error};
         mbar_wait(&bar, 0, g, 31);
     }
 }

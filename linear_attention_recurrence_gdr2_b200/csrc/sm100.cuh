@@ -71,19 +71,23 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
 // Shared state of the bounded waits of one CTA: the first wait that runs out
 // of time records where it gave up and every later wait returns at once.
 struct WaitGuard {
-    uint64_t deadline_ns;      // absolute %globaltimer deadline
+    uint64_t timeout_ns;       // limit of one wait, from its first unsuccessful probe
     volatile int *abort_flag;  // in shared memory: nonzero once any wait timed out
     int *error_word;           // global: receives the first error code
 };
 
 // Waits for phase `parity` of `bar`; returns false if the CTA is aborting or
-// the deadline passes (then the abort flag and the global error word are set).
+// the time limit passes (then the abort flag and the global error word are
+// set). A phase that has already completed costs one probe: the timer is
+// read only once the first probe fails.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitGuard &g,
                                           int site) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t deadline = globaltimer_ns() + g.timeout_ns;
     uint32_t spins = 0;
     while (!mbar_try(bar, parity)) {
         if (*g.abort_flag) return false;
-        if ((++spins & 7u) == 0 && globaltimer_ns() > g.deadline_ns) {
+        if ((++spins & 7u) == 0 && globaltimer_ns() > deadline) {
             *g.abort_flag = 1;
             atomicCAS(g.error_word, 0, 0x100 | site);
             return false;

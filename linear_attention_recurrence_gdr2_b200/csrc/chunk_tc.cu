@@ -747,12 +747,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     }
                     tmem_st16(tb + kTmSB + lane_off + 32 * hh, s0b);
                     tmem_st16(tb + kTmSB + lane_off + 32 * hh + 16, s1b);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
                     tc_wait_st();
                     tc_fence_before();
                     named_bar_sync(kBarEpi, 128);
                     if (te == 0) mbar_arrive(&bars[hh ? M_SREADY_HI : M_SREADY_LO]);
+                    // the fp32 master: first read again by the next chunk's update MMAs,
+                    // which wait for the U hand-off (its tc_wait_st covers these stores)
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
                 } else if (prm.final_state) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) {
@@ -784,6 +786,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             named_bar_sync(kBarEpi, 128);
             if (te == 0) mbar_arrive(&bars[M_OFULL]);
         }
+        tc_wait_st();  // (a master write-back may still be in flight after an abort)
     }
     } else {
     // =========================================================================

@@ -284,12 +284,17 @@ def main():
     B, T, H, d = inp.q.shape
     o = torch.empty((B, T, H, d), dtype=tdt, device=dev)
     sf = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    dcode = gdr2.GDR2_BF16 if inp.dtype == "bf16" else gdr2.GDR2_FP32
+    ws_bytes = gdr2.workspace_size(B, T, H, d, d, N, dcode)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
     def step():
         gdr2.chunk_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["log_alpha"], dv_["b"], dv_["w"], s0, cu,
-                       o=o, final_state=sf)
+                       o=o, final_state=sf, workspace=ws)
 
-    launches_per_step = 1
+    # the chunk kernel; plus the order kernel of a packed batch, or the combine
+    # and correction kernels of a segment split (few long sequences)
+    launches_per_step = 1 + (1 if cu is not None and N > 1 else 0) + (2 if cu is None and ws_bytes > 0 else 0)
     clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     with clocks:
         for _ in range(args.warmup):

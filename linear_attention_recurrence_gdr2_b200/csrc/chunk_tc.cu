@@ -67,7 +67,7 @@ __device__ int g_chunk_tc_error;
 __device__ unsigned long long *g_chunk_tc_trace;
 #define GDR2_TRACE_AT(chunk, ev)                                                                \
     do {                                                                                        \
-        const unsigned ts_ = blockIdx.x < 4 ? blockIdx.x : blockIdx.x - 16;                     \
+        const unsigned ts_ = blockIdx.x < 4 ? blockIdx.x : (blockIdx.x - 20u < 4u ? blockIdx.x - 16u : 8u); \
         if (ts_ < 8 && g_chunk_tc_trace && (chunk) < 1024)                                      \
             g_chunk_tc_trace[((size_t)ts_ * 1024 + (chunk)) * 32 + (ev)] = clock64();           \
     } while (0)
@@ -164,6 +164,14 @@ struct TcParams {
     __nv_bfloat16 *o;
     float *final_state;
     int64_t T, H, units;
+    // segment-parallel scan (nseg > 1): per sequence, jobs 0..nseg-1 run the
+    // segments from their entry state (the true one for segment 0, else 0) and
+    // write o and seg_s0; jobs nseg..2 nseg-2 run segments 1..nseg-1 from the
+    // identity with z = 0 and write psi and seg_phi
+    int nseg;
+    int64_t seg_len;
+    __nv_bfloat16 *psi;
+    float *seg_s0, *seg_phi;
 };
 
 // Bounded wait on a barrier of this CTA (CTA-scope acquire: the peer's
@@ -318,10 +326,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     const int64_t H = prm.H;
     const int64_t unit = (int64_t)(blockIdx.x / (2 * kPairs)) * kPairs + (rank % kPairs);
     const bool valid = unit < prm.units;  // the last cluster may hold a padding pair
+    const int jobs = 2 * prm.nseg - 1;    // per (sequence, head)
     int64_t h = 0, n = 0, t_begin = 0, t_end = 0;
+    int job = 0;
     if (valid) {
         h = unit % H;
-        n = prm.order ? (int64_t)prm.order[unit / H] : (int64_t)(unit / H);
+        const int64_t nj = unit / H;
+        job = (int)(nj % jobs);
+        n = prm.order ? (int64_t)prm.order[nj / jobs] : (int64_t)(nj / jobs);
         if (prm.cu_seqlens) {
             t_begin = prm.cu_seqlens[n];
             t_end = prm.cu_seqlens[n + 1];
@@ -330,15 +342,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             t_end = t_begin + prm.T;
         }
     }
+    // segment of this job, and whether it is an identity-state run with z = 0
+    const bool zero_v = job >= prm.nseg;
+    const int seg = zero_v ? job - prm.nseg + 1 : job;
+    if (prm.nseg > 1 && valid) {
+        const int64_t sb = t_begin + seg * prm.seg_len;
+        t_end = sb + prm.seg_len < t_end ? sb + prm.seg_len : t_end;
+        t_begin = sb;
+    }
     const int nc = (int)((t_end - t_begin + 63) / 64);
     const int64_t state_base = (n * H + h) * (int64_t)kD * kD;
+    // entry state (null: zero, unless identity) and where the exit state goes
+    const float *init_ptr = nullptr;
+    float *final_ptr = nullptr;
+    if (prm.nseg == 1) {
+        init_ptr = prm.init_state ? prm.init_state + state_base : nullptr;
+        final_ptr = prm.final_state ? prm.final_state + state_base : nullptr;
+    } else {
+        const int64_t seg_base = ((n * prm.nseg + seg) * H + h) * (int64_t)kD * kD;
+        init_ptr = (!zero_v && seg == 0 && prm.init_state) ? prm.init_state + state_base : nullptr;
+        final_ptr = (zero_v ? prm.seg_phi : prm.seg_s0) + seg_base;
+    }
 
     if (nc == 0) {
         // empty sequence (both CTAs of the pair are here): the final state is
         // the initial state; then only the cluster's three barriers are joined
-        if (valid && is_main && prm.final_state)
+        if (valid && is_main && final_ptr)
             for (int i = tid; i < kD * kD; i += kThreadsTC)
-                prm.final_state[state_base + i] = prm.init_state ? prm.init_state[state_base + i] : 0.f;
+                final_ptr[i] = init_ptr ? init_ptr[i] : 0.f;
         cluster_sync_all();
         cluster_sync_all();
         cluster_sync_all();
@@ -397,20 +428,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             int wissued = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                if (c >= 2 && !wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
-                    break;
-                const int z = (int)(t_begin + 64 * c);
-                GDR2_TRACE_AT(c, 0);
-                mbar_arrive_expect_tx(&bars[M_VFULL0 + s], 16384);
-                for (int blk = 0; blk < 2; ++blk)
-                    tma_load_3d(smem + mZ(s) + blk * 8192, &map_v, &bars[M_VFULL0 + s], 64 * blk, (int)h, z);
-                (s ? vissued1 : vissued0) = (c >> 1) + 1;
-                // the single w buffer: free once Z of chunk c-1 is done
-                if (c >= 1 && !wait_bar(&bars[M_WTFREE], (c - 1) & 1, abort_flag, peer_abort, 4)) break;
-                mbar_arrive_expect_tx(&bars[M_WTFULL], 16384);
-                for (int blk = 0; blk < 2; ++blk)
-                    tma_load_3d(smem + kM_WT + blk * 8192, &map_w, &bars[M_WTFULL], 64 * blk, (int)h, z);
-                ++wissued;
+                if (!zero_v) {  // (an identity run with z = 0 loads neither)
+                    if (c >= 2 && !wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
+                        break;
+                    const int z = (int)(t_begin + 64 * c);
+                    GDR2_TRACE_AT(c, 0);
+                    mbar_arrive_expect_tx(&bars[M_VFULL0 + s], 16384);
+                    for (int blk = 0; blk < 2; ++blk)
+                        tma_load_3d(smem + mZ(s) + blk * 8192, &map_v, &bars[M_VFULL0 + s], 64 * blk, (int)h, z);
+                    (s ? vissued1 : vissued0) = (c >> 1) + 1;
+                    // the single w buffer: free once Z of chunk c-1 is done
+                    if (c >= 1 && !wait_bar(&bars[M_WTFREE], (c - 1) & 1, abort_flag, peer_abort, 4)) break;
+                    mbar_arrive_expect_tx(&bars[M_WTFULL], 16384);
+                    for (int blk = 0; blk < 2; ++blk)
+                        tma_load_3d(smem + kM_WT + blk * 8192, &map_w, &bars[M_WTFULL], 64 * blk, (int)h, z);
+                    ++wissued;
+                }
                 // slot s of chunk c - 2 fully consumed (its last MMA is done):
                 // the helper may copy chunk c into it
                 if (c >= 2) {
@@ -527,6 +560,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
+            if (zero_v) {
+                // Z = 0: clear the slot once its previous U0 MMA is done (that wait
+                // also paces the hand-offs, one phase per chunk and slot)
+                if (!group_and(kBarZ, 128, c < 2 || wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag,
+                                                               peer_abort, 5)))
+                    break;
+                if (c < 2) {
+                    uint4 *zt = reinterpret_cast<uint4 *>(smem + mZ(s));
+                    for (int i = tp; i < 16384 / 16; i += 128) zt[i] = make_uint4(0u, 0u, 0u, 0u);
+                    fence_proxy_async_smem();
+                }
+                named_bar_sync(kBarZ, 128);
+                if (tp == 0) mbar_arrive(&bars[M_ZREADY0 + s]);
+                continue;
+            }
             if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5) &&
                                            wait_bar(&bars[M_WTFULL], c & 1, abort_flag, peer_abort, 6)))
                 break;
@@ -562,6 +610,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int pw = warp - 8, tp = tid - 256;
         const int rrow = 16 * pw + (lane & 15), kb = lane >> 4;
         const uint32_t h_tfree = mapa_shared(smem_u32(&bars[H_TFREE0]), peer);
+        __nv_bfloat16 *obase = zero_v ? prm.psi : prm.o;  // (an identity run writes psi)
         // o of chunk cc from the staging tile: 16-byte pieces, 16 per row; rows
         // past the sequence end are not written
         auto store_o = [&](int cc) -> bool {
@@ -573,7 +622,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const int idx = tp + 128 * i, r = idx >> 4, piece = idx & 15;
                 if (r < L) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(smem + kM_OST + r * kOPitch + 16 * piece);
-                    *reinterpret_cast<uint4 *>(prm.o + ((t0 + r) * H + h) * kD + 8 * piece) = v;
+                    *reinterpret_cast<uint4 *>(obase + ((t0 + r) * H + h) * kD + 8 * piece) = v;
                 }
             }
             named_bar_sync(kBarW, 128);
@@ -634,7 +683,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int ch = 32 * g4 + q;
-                    const float s0 = prm.init_state ? prm.init_state[state_base + (int64_t)ch * kD + j] : 0.f;
+                    const float s0 = init_ptr ? init_ptr[(int64_t)ch * kD + j] : (zero_v && ch == j ? 1.f : 0.f);
                     m[q] = __float_as_uint(vecF[ch] * s0);
                 }
 #pragma unroll
@@ -755,11 +804,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     // which wait for the U hand-off (its tc_wait_st covers these stores)
                     tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
                     tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
-                } else if (prm.final_state) {
+                } else if (final_ptr) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) {
-                        prm.final_state[state_base + (int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
-                        prm.final_state[state_base + (int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
+                        final_ptr[(int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
+                        final_ptr[(int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
                     }
                 }
             }
@@ -1253,7 +1302,8 @@ bool chunk_tc_supported(const ChunkArgs &a)
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
     const int64_t tokens = a.B * a.T;
-    const int64_t units = a.num_seqs * a.H;  // two CTAs per (sequence, head), kPairs pairs per cluster
+    // two CTAs per job, kPairs pairs per cluster; 2 nseg - 1 jobs per (sequence, head)
+    const int64_t units = a.num_seqs * a.H * (2 * (int64_t)a.nseg - 1);
     if (units == 0) return cudaSuccess;
     const int64_t clusters = (units + kPairs - 1) / kPairs;
     if (tokens > 0x7fffffffLL || 2 * kPairs * clusters > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -1278,6 +1328,12 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.T = a.T;
     p.H = a.H;
     p.units = units;
+    p.nseg = a.nseg;
+    p.seg_len = a.seg_len;
+    unsigned char *ws = static_cast<unsigned char *>(a.seg_ws);
+    p.psi = a.nseg > 1 ? reinterpret_cast<__nv_bfloat16 *>(ws + seg_psi_offset()) : nullptr;
+    p.seg_s0 = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_state_offset(a.B, a.T, a.H)) : nullptr;
+    p.seg_phi = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_phi_offset(a.B, a.T, a.H, a.nseg)) : nullptr;
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;

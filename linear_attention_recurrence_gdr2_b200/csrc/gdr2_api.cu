@@ -23,6 +23,23 @@ gdr2_status check_dims(int64_t d_k, int64_t d_v)
 
 }  // namespace
 
+namespace gdr2 {
+
+gdr2_status chunk_fwd_min_workspace(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                    int64_t num_seqs, gdr2_dtype dtype, size_t *bytes)
+{
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    // A packed batch of several sequences (the only case with num_seqs != B)
+    // needs room for its longest-first processing order.
+    *bytes = (B == 1 && num_seqs > 1) ? order_bytes(num_seqs) : 0;
+    return GDR2_OK;
+}
+
+}  // namespace gdr2
+
 extern "C" {
 
 const char *gdr2_status_string(gdr2_status s)
@@ -45,13 +62,15 @@ gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H, int64
                                           size_t *bytes)
 {
     if (!bytes) return GDR2_ERR_INVALID_ARG;
-    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
-    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
-    gdr2_status st = check_dims(d_k, d_v);
+    size_t min_bytes = 0;
+    gdr2_status st = gdr2::chunk_fwd_min_workspace(B, T, H, d_k, d_v, num_seqs, dtype, &min_bytes);
     if (st != GDR2_OK) return st;
-    // A packed batch of several sequences (the only case with num_seqs != B)
-    // needs room for its longest-first processing order.
-    *bytes = (B == 1 && num_seqs > 1) ? gdr2::order_bytes(num_seqs) : 0;
+    // A packed batch of several sequences needs its processing order; a
+    // fixed-length batch of few long sequences may use the segment split.
+    *bytes = (B == 1 && num_seqs > 1)
+                 ? min_bytes
+                 : gdr2::plan_segments(B, T, H, d_k, dtype == GDR2_BF16).ws_bytes;
+    if (*bytes < min_bytes) *bytes = min_bytes;
     return GDR2_OK;
 }
 
@@ -82,11 +101,17 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     if (final_state && !aligned16(final_state)) return GDR2_ERR_INVALID_ARG;
     if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDR2_ERR_INVALID_ARG;
     size_t need = 0;
-    st = gdr2_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, dtype, &need);
+    st = gdr2::chunk_fwd_min_workspace(B, T, H, d_k, d_v, num_seqs, dtype, &need);
     if (st != GDR2_OK) return st;
     if (need > 0 && (!workspace || workspace_bytes < need)) return GDR2_ERR_WORKSPACE;
-    if (need > 0 && !aligned16(workspace)) return GDR2_ERR_INVALID_ARG;
+    if ((need > 0 || workspace_bytes > 0) && workspace && !aligned16(workspace)) return GDR2_ERR_INVALID_ARG;
     if (num_seqs == 0) return GDR2_OK;
+    // segment split when the workspace holds it (fixed-length bf16 batches only)
+    gdr2::SegPlan plan{1, 0, 0};
+    if (!cu_seqlens) {
+        plan = gdr2::plan_segments(B, T, H, d_k, dtype == GDR2_BF16);
+        if (plan.nseg > 1 && (!workspace || workspace_bytes < plan.ws_bytes)) plan = gdr2::SegPlan{1, 0, 0};
+    }
 
     gdr2::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.b = b; a.w = w;
@@ -98,6 +123,9 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.num_seqs = num_seqs;
     a.bf16 = dtype == GDR2_BF16;
+    a.nseg = plan.nseg;
+    a.seg_len = plan.seg_len;
+    a.seg_ws = plan.nseg > 1 ? workspace : nullptr;
     cudaError_t e = cudaSuccess;
     if (cu_seqlens && num_seqs > 1) {
         a.order = static_cast<const int32_t *>(workspace);
@@ -105,8 +133,12 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
                                          (cudaStream_t)stream);
         if (e != cudaSuccess) return GDR2_ERR_CUDA;
     }
-    e = gdr2::chunk_tc_supported(a) ? gdr2::launch_chunk_tc(a, (cudaStream_t)stream)
-                                                : gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
+    if (gdr2::chunk_tc_supported(a)) {
+        e = gdr2::launch_chunk_tc(a, (cudaStream_t)stream);
+        if (e == cudaSuccess && a.nseg > 1) e = gdr2::launch_segment_fix(a, (cudaStream_t)stream);
+    } else {
+        e = gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
+    }
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 

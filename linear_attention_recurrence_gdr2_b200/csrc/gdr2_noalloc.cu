@@ -51,8 +51,8 @@ extern "C" gdr2_status gdr2_chunk_fwd_noalloc(const void *q, const void *k, cons
                                               int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
                                               void *o, float *final_state, void *stream)
 {
-    size_t need = 0;
-    gdr2_status st = gdr2_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, dtype, &need);
+    size_t need = 0;  // (without the optional segment split, which needs far more)
+    gdr2_status st = gdr2::chunk_fwd_min_workspace(B, T, H, d_k, d_v, num_seqs, dtype, &need);
     if (st != GDR2_OK) return st;
     if (need > kNoAllocScratchBytes) return GDR2_ERR_UNSUPPORTED;  // more sequences than the array holds
     void *scratch = nullptr;

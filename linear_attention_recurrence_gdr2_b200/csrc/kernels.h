@@ -4,7 +4,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/gdr2.h"
+
 namespace gdr2 {
+
+// Workspace a chunk forward cannot run without (the packed-batch order); the
+// public size query adds the optional segment split on top.
+gdr2_status chunk_fwd_min_workspace(int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                                    int64_t num_seqs, gdr2_dtype dtype, size_t *bytes);
 
 struct DecodeArgs {
     const void *q, *k, *v, *b, *w;
@@ -25,7 +32,31 @@ struct ChunkArgs {
     float *final_state;        // may be null
     int64_t B, T, H, dk, dv, num_seqs;
     bool bf16;
+    // Segment-parallel scan (fixed-length bf16 batches of few long sequences;
+    // see segments.cu): nseg segments of seg_len tokens per sequence, scratch
+    // in seg_ws. nseg == 1: one serial pass per (sequence, head).
+    int nseg = 1;
+    int64_t seg_len = 0;
+    void *seg_ws = nullptr;
 };
+
+// Segment plan of the tensor-core chunk forward: how many segments each
+// sequence of a fixed-length batch is split into (1 = none), and the scratch
+// the split needs.
+struct SegPlan {
+    int nseg;
+    int64_t seg_len;   // tokens per segment (a multiple of 64)
+    size_t ws_bytes;   // psi (tokens x H x 128 bf16) + two [N][nseg][H][128][128] fp32 arrays
+};
+SegPlan plan_segments(int64_t B, int64_t T, int64_t H, int64_t d, bool bf16);
+// Byte offsets inside the segment scratch.
+size_t seg_psi_offset();
+size_t seg_state_offset(int64_t B, int64_t T, int64_t H);
+size_t seg_phi_offset(int64_t B, int64_t T, int64_t H, int nseg);
+
+// After the segmented chunk forward: chain the segment states, write the
+// final states and add each later segment's entry-state contribution to o.
+cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 

@@ -82,7 +82,7 @@ struct WaitGuard {
 // read only once the first probe fails.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitGuard &g,
                                           int site) {
-    if (mbar_try(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;  // (non-blocking probe first: often already complete)
     const uint64_t deadline = globaltimer_ns() + g.timeout_ns;
     uint32_t spins = 0;
     while (!mbar_try(bar, parity)) {

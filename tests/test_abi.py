@@ -112,10 +112,27 @@ def test_recurrent_step_rejects_bad_arguments(over, expect):
 def test_packed_batch_needs_workspace():
     need = gdr2.workspace_size(1, 1000, 4, 128, 128, 3, gdr2.GDR2_BF16)
     assert need >= 3 * 4 and need % 256 == 0
-    assert gdr2.workspace_size(2, 1000, 4, 128, 128, 2, gdr2.GDR2_BF16) == 0
+    # fixed-length batches need none; many (sequence, head) units get no split
+    assert gdr2.workspace_size(4, 2048, 16, 128, 128, 4, gdr2.GDR2_BF16) == 0
+    assert gdr2.workspace_size(2, 1000, 4, 128, 128, 2, gdr2.GDR2_FP32) == 0
     assert _chunk(B=1, N=3, cu=FAKE) == WORKSPACE
     assert _chunk(B=1, N=3, cu=FAKE, ws=FAKE, wsb=need - 1) == WORKSPACE
     assert _chunk(B=1, N=3, cu=FAKE, ws=FAKE + 8, wsb=need) == INVALID  # misaligned workspace
+
+
+def test_segment_split_workspace():
+    """Few long bf16 sequences report room for the segment-parallel scan: o-sized
+    psi (bf16) plus two [N][segments][H][128][128] fp32 state arrays."""
+    B, T, H = 1, 32768, 16
+    need = gdr2.workspace_size(B, T, H, 128, 128, B, gdr2.GDR2_BF16)
+    psi = B * T * H * 128 * 2
+    assert need >= psi + 2 * 2 * B * H * 128 * 128 * 4  # at least two segments
+    assert need % 256 == 0
+    # no split for d = 64, fp32, or sequences too short for two 8-chunk segments
+    assert gdr2.workspace_size(B, T, H, 64, 64, B, gdr2.GDR2_BF16) == 0
+    assert gdr2.workspace_size(B, T, H, 128, 128, B, gdr2.GDR2_FP32) == 0
+    assert gdr2.workspace_size(1, 64 * 15, 1, 128, 128, 1, gdr2.GDR2_BF16) == 0
+    assert gdr2.workspace_size(1, 64 * 16, 1, 128, 128, 1, gdr2.GDR2_BF16) > 0
 
 
 def test_empty_problems_return_ok_without_launch():

@@ -129,6 +129,42 @@ def test_chunk_strong_decay_in_range(cuda_device):
     check_full(inp, cuda_device, "strong decay")
 
 
+@pytest.mark.parametrize("B,T,H,la_scale,init", [
+    (1, 2048, 2, 0.01, 0.05),    # 4 segments of 512 tokens, nonzero initial state
+    (2, 1000, 3, 0.02, None),    # 2 segments, ragged last chunk
+    (1, 8192, 1, 0.005, 0.02),   # 16 segments: the longest combine chain
+])
+def test_chunk_segment_split(cuda_device, B, T, H, la_scale, init):
+    """Few long bf16 sequences run as concurrent segments (from the segment's
+    entry state 0, or the true one for the first; and from the identity with
+    z = 0), then the affine combine of the segment states and the o
+    correction. Weak decay keeps each segment's entry state influential.
+    Every element against the oracle."""
+    assert gdr2().workspace_size(B, T, H, 128, 128, B, gdr2().GDR2_BF16) > 0  # split in use
+    inp = gen.make_inputs(B, T, H, 128, 128, "bf16", seed=11, la_scale=la_scale, init_std=init)
+    check_full(inp, cuda_device, f"segments B{B} T{T} H{H}")
+
+
+def test_chunk_segment_split_matches_serial_scan(cuda_device):
+    """The split and the serial scan (the allocation-free entry point never
+    splits) agree with each other as well as with the oracle."""
+    import torch
+    inp = gen.make_inputs(1, 2048, 2, 128, 128, "bf16", seed=12, la_scale=0.01, init_std=0.05)
+    o_split, s_split = run_chunk(inp, cuda_device)
+    t = upload(inp, cuda_device)
+    o2 = torch.empty_like(t["v"])
+    s2 = torch.empty_like(t["init_state"])
+    gdr2().chunk_fwd_noalloc(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"],
+                             t["init_state"], t["cu_seqlens"], o=o2, final_state=s2)
+    torch.cuda.synchronize()
+    o_r, s_r = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w, inp.init_state)
+    assert_close("serial o", to_np(o2), o_r, "bf16")
+    assert_close("serial state", to_np(s2), s_r, "bf16")
+    assert_close("split o", o_split, o_r, "bf16")
+    assert_close("split state", s_split, s_r, "bf16")
+    assert rel_l2(o_split, to_np(o2)) < TOL["bf16"] and rel_l2(s_split, to_np(s2)) < TOL["bf16"]
+
+
 @pytest.mark.slow
 def test_layer_prefill_full_size(cuda_device):
     """B=4, H=16, T=2048, d=128, bf16: six (sequence, head) units recomputed."""

@@ -112,12 +112,18 @@ int gdr2_version(void);
  *                may alias init_state (each head reads its initial state
  *                before it writes its final state)
  *   workspace, workspace_bytes
- *                device scratch of at least gdr2_chunk_fwd_workspace_size()
- *                bytes, 16-byte aligned (NULL allowed when that size is 0).
- *                A packed batch of several sequences uses it for the order in
- *                which sequences are processed (longest first, computed on the
- *                device from cu_seqlens); its contents are overwritten, so
- *                calls that share a workspace must be ordered on the GPU.
+ *                device scratch, 16-byte aligned. A packed batch of several
+ *                sequences requires the size gdr2_chunk_fwd_workspace_size()
+ *                reports: the order in which sequences are processed (longest
+ *                first, computed on the device from cu_seqlens). A fixed-length
+ *                bf16 batch with d = 128 and few (sequence, head) units may be
+ *                given the (larger) reported size to run the segment-parallel
+ *                scan: each sequence is cut into segments that run concurrently
+ *                (from zero and from the identity state), then the segment
+ *                states are chained in fp32 and the later segments' outputs
+ *                corrected; with less (down to NULL / 0) it runs the serial
+ *                scan. Contents are overwritten, so calls that share a
+ *                workspace must be ordered on the GPU.
  *   stream       cudaStream_t
  * Precision: with GDR2_FP32 every product runs in fp32 on CUDA cores; with
  * GDR2_BF16 the dense intra-chunk contractions run on the tensor cores with
@@ -131,9 +137,13 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v,
                            void *o, float *final_state, void *workspace,
                            size_t workspace_bytes, void *stream);
 
-/* Scratch bytes gdr2_chunk_fwd needs for this problem (written to *bytes):
- * 0 for fixed-length batches; a small multiple of 256 bytes (4 bytes per
- * sequence) for a packed batch of num_seqs > 1 sequences (B == 1). */
+/* Scratch bytes gdr2_chunk_fwd uses for this problem (written to *bytes), a
+ * multiple of 256: for a packed batch of num_seqs > 1 sequences (B == 1), 4
+ * bytes per sequence (required); for a fixed-length batch, 0 or, when the
+ * segment-parallel scan applies (bf16, d = 128, at most 64 / (2P - 1) (sequence,
+ * head) units for P >= 2 segments of >= 8 chunks), B*T*H*256 bytes (the
+ * per-token readout maps, bf16) plus 2 * B*P*H*64 KiB (segment states, fp32)
+ * (optional: a smaller workspace runs the serial scan). */
 gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
                                           int64_t d_k, int64_t d_v,
                                           int64_t num_seqs, gdr2_dtype dtype,
@@ -154,7 +164,8 @@ gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
  * loads the library until the process exits.
  *   - Limit: a packed batch (cu_seqlens, num_seqs > 1) may hold at most 16384
  *     sequences; larger ones return GDR2_ERR_UNSUPPORTED before any launch.
- *     Fixed-length batches use no scratch and have no extra limit.
+ *     Fixed-length batches use no scratch and have no extra limit (they run
+ *     the serial scan, never the segment-parallel one).
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.

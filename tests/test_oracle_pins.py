@@ -10,6 +10,7 @@ import pytest
 
 import oracle
 import pins
+from linear_attention_recurrence_gdr2_b200 import inputs as gen
 
 
 def oracle_fwd(q, k, v, la, b, w, s0=None, cu=None):
@@ -138,3 +139,33 @@ def test_planted_mistake_is_caught(mutation):
     fwd = lambda *a, **kw: loop_forward(*a, mutation=mutation, **kw)
     step = lambda *a, **kw: loop_step(*a, mutation=mutation, **kw)
     assert _run_all_pins(fwd, step), f"no pin caught mutation {mutation!r}"
+
+
+def test_segment_split_identity():
+    """The segment-parallel scan's decomposition, on the oracle alone (fp64):
+    running each segment from a zero state, and from the identity with z = 0
+    (giving its transition Phi and readout map psi_t = Phi_t^T q_t), then
+    chaining S_start(p+1) = Phi_p S_start(p) + S0_p and adding S_start^T psi_t,
+    reproduces one serial run (the affine structure of the rule)."""
+    inp = gen.make_inputs(2, 300, 2, 16, 16, "fp32", seed=31, la_scale=0.01, init_std=0.1)
+    o_ref, s_ref = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w, inp.init_state)
+    L, T = 128, 300
+    eye = np.broadcast_to(np.eye(16, dtype=np.float32), inp.init_state.shape).copy()
+    o = np.zeros_like(o_ref)
+    s_start = inp.init_state.astype(np.float64)
+    for p0 in range(0, T, L):
+        sl = slice(p0, min(p0 + L, T))
+        cut = lambda x: np.ascontiguousarray(x[:, sl])
+        zero = np.zeros_like(inp.init_state)
+        o_a, s_a = oracle.forward(cut(inp.q), cut(inp.k), cut(inp.v), cut(inp.log_alpha), cut(inp.b),
+                                  cut(inp.w), inp.init_state if p0 == 0 else zero)
+        o_b, phi = oracle.forward(cut(inp.q), cut(inp.k), np.zeros_like(cut(inp.v)), cut(inp.log_alpha),
+                                  cut(inp.b), cut(inp.w), eye)
+        if p0 == 0:
+            o[:, sl] = o_a
+            s_start = s_a
+        else:
+            o[:, sl] = o_a + np.einsum("ntha,nhab->ntbh", o_b, s_start).transpose(0, 1, 3, 2)
+            s_start = np.einsum("nhik,nhkj->nhij", phi, s_start) + s_a
+    assert np.max(np.abs(o - o_ref)) < 1e-12 * max(1.0, np.max(np.abs(o_ref)))
+    assert np.max(np.abs(s_start - s_ref)) < 1e-12 * max(1.0, np.max(np.abs(s_ref)))

@@ -204,6 +204,47 @@ gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
                                 gdr2_dtype dtype, void *o, void *stream);
 
 /*
+ * Fused prologue (bit flags for the *_preact entry points below).
+ *
+ * In the Gated DeltaNet-2 block ("Block design and hybrid model", ainews
+ * article) the query and key paths end in L2 normalisation, the erase and write
+ * gates are sigmoid projections and the decay comes from its own linear
+ * branch. These flags let the kernels apply those last element-wise steps to
+ * pre-activation inputs while loading them, instead of a separate pass over
+ * the five tensors. Each is computed in fp32 per token and head:
+ *   GDR2_PROLOGUE_QK_L2NORM      q, k <- x / sqrt(sum_c x_c^2 + 1e-6)
+ *   GDR2_PROLOGUE_GATE_SIGMOID   b, w <- 1 / (1 + exp(-x))
+ *   GDR2_PROLOGUE_DECAY_SOFTPLUS log_alpha <- -softplus(x) = -log(1 + exp(x))
+ * (the pages do not print the decay branch's activation; -softplus is the
+ * usual way to map a projection to a log-decay <= 0, and is this library's
+ * reading). v passes unchanged: its SiLU precedes the operator.
+ */
+#define GDR2_PROLOGUE_QK_L2NORM 1u
+#define GDR2_PROLOGUE_GATE_SIGMOID 2u
+#define GDR2_PROLOGUE_DECAY_SOFTPLUS 4u
+
+/* gdr2_chunk_fwd on pre-activation inputs: the `prologue` flags (a combination
+ * of GDR2_PROLOGUE_*) name the activations applied to q, k, b, w, log_alpha on
+ * load; everything else (arguments, layouts, workspace, errors) is exactly as
+ * for gdr2_chunk_fwd, which equals this call with prologue = 0. Unknown flag
+ * bits return GDR2_ERR_INVALID_ARG. */
+gdr2_status gdr2_chunk_fwd_preact(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const void *b, const void *w,
+                                  const float *init_state, const int32_t *cu_seqlens,
+                                  int64_t B, int64_t T, int64_t H, int64_t d_k,
+                                  int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                                  void *o, float *final_state, void *workspace,
+                                  size_t workspace_bytes, uint32_t prologue, void *stream);
+
+/* gdr2_recurrent_step on pre-activation inputs (same `prologue` flags). */
+gdr2_status gdr2_recurrent_step_preact(const void *q, const void *k, const void *v,
+                                       const float *log_alpha, const void *b,
+                                       const void *w, float *state, int64_t N,
+                                       int64_t H, int64_t d_k, int64_t d_v,
+                                       gdr2_dtype dtype, void *o, uint32_t prologue,
+                                       void *stream);
+
+/*
  * gdr2_check_device_error -- reports whether a kernel of this library gave up
  * a bounded device-side wait on the current device since the last check.
  *

@@ -25,6 +25,11 @@ LIB_PATH = os.path.join(_HERE, "libgdr2.so")
 GDR2_OK = 0
 GDR2_FP32 = 0
 GDR2_BF16 = 1
+# fused prologue flags (gdr2.h)
+GDR2_PROLOGUE_QK_L2NORM = 1
+GDR2_PROLOGUE_GATE_SIGMOID = 2
+GDR2_PROLOGUE_DECAY_SOFTPLUS = 4
+GDR2_PROLOGUE_ALL = 7
 
 _lock = threading.Lock()
 _lib = None
@@ -74,6 +79,15 @@ def lib() -> ctypes.CDLL:
             L.gdr2_recurrent_step.argtypes = [
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                 _i64, _i64, _i64, _i64, ctypes.c_int, _vp, _vp]
+            L.gdr2_chunk_fwd_preact.restype = ctypes.c_int
+            L.gdr2_chunk_fwd_preact.argtypes = [
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
+                _vp, _vp, _vp, ctypes.c_size_t, ctypes.c_uint32, _vp]
+            L.gdr2_recurrent_step_preact.restype = ctypes.c_int
+            L.gdr2_recurrent_step_preact.argtypes = [
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                _i64, _i64, _i64, _i64, ctypes.c_int, _vp, ctypes.c_uint32, _vp]
             _lib = L
     return _lib
 
@@ -137,12 +151,15 @@ def workspace_size(B: int, T: int, H: int, d_k: int, d_v: int, num_seqs: int,
 
 def chunk_fwd(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None, *,
               o=None, final_state=None, output_final_state: bool = True,
-              workspace=None, stream=None) -> Tuple["torch.Tensor", Optional["torch.Tensor"]]:
+              workspace=None, prologue: int = 0,
+              stream=None) -> Tuple["torch.Tensor", Optional["torch.Tensor"]]:
     """Chunkwise forward of Gated Delta Rule-2 (see gdr2_chunk_fwd in gdr2.h).
 
     q, k, b: [B, T, H, d_k]; v, w: [B, T, H, d_v] (bf16 or fp32, all alike);
     log_alpha: [B, T, H, d_k] fp32; init_state: [N, H, d_k, d_v] fp32 or None;
     cu_seqlens: int32 [N+1] on the device (then B == 1) or None.
+    prologue: GDR2_PROLOGUE_* flags (gdr2_chunk_fwd_preact): activations the
+    kernels apply to pre-activation q, k, b, w, log_alpha on load.
     Returns (o [B, T, H, d_v], final_state [N, H, d_k, d_v] fp32 or None).
     """
     import torch
@@ -177,6 +194,14 @@ def chunk_fwd(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None, *,
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if prologue:
+        st = lib().gdr2_chunk_fwd_preact(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(init_state),
+            _ptr(cu_seqlens), B, T, H, dk, dv, N, code, _ptr(o), _ptr(final_state),
+            _ptr(workspace), ws_bytes, int(prologue), _stream_handle(stream))
+        if st != GDR2_OK:
+            raise GDR2Error("gdr2_chunk_fwd_preact", st)
+        return o, final_state
     st = lib().gdr2_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(init_state),
         _ptr(cu_seqlens), B, T, H, dk, dv, N, code, _ptr(o), _ptr(final_state),
@@ -215,11 +240,12 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None
     return o, final_state
 
 
-def recurrent_step(q, k, v, log_alpha, b, w, state, *, o=None, stream=None):
+def recurrent_step(q, k, v, log_alpha, b, w, state, *, o=None, prologue: int = 0, stream=None):
     """One decode step (see gdr2_recurrent_step in gdr2.h); state updated in place.
 
     q, k, b: [N, H, d_k]; v, w: [N, H, d_v] (bf16 or fp32, all alike);
     log_alpha: [N, H, d_k] fp32; state: [N, H, d_k, d_v] fp32. Returns o [N, H, d_v].
+    prologue: GDR2_PROLOGUE_* flags (gdr2_recurrent_step_preact).
     """
     import torch
     dev = q.device
@@ -237,6 +263,13 @@ def recurrent_step(q, k, v, log_alpha, b, w, state, *, o=None, stream=None):
         o = torch.empty((N, H, dv), dtype=dt, device=dev)
     else:
         _check(o, "o", (N, H, dv), dt, dev)
+    if prologue:
+        st = lib().gdr2_recurrent_step_preact(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(state),
+            N, H, dk, dv, code, _ptr(o), int(prologue), _stream_handle(stream))
+        if st != GDR2_OK:
+            raise GDR2Error("gdr2_recurrent_step_preact", st)
+        return o
     st = lib().gdr2_recurrent_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(state),
         N, H, dk, dv, code, _ptr(o), _stream_handle(stream))

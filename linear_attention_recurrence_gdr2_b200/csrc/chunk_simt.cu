@@ -46,9 +46,12 @@ struct SimtSmem {
     float z[kChunk][kDVT]; // z -> r = z - Ebar S0 -> u (in place)
     float gC[DK];
     float gm[DK];
+    float qinv[kChunk];    // prologue: 1 / ||q_r||, 1 / ||k_r|| (1 without it)
+    float kinv[kChunk];
 };
 
-template <typename Tin, int DK>
+// kPre: the fused prologue is compiled in (the *_preact calls only).
+template <typename Tin, int DK, bool kPre>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_simt_kernel(ChunkArgs args)
 {
@@ -82,9 +85,36 @@ chunk_simt_kernel(ChunkArgs args)
         sm.s0[c][j] = args.init_state ? args.init_state[state_off + (int64_t)c * DV + j] : 0.f;
     }
 
+    const uint32_t pre = kPre ? args.pre : 0u;
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kChunk) {
         const int L = (int)(t_end - t0 < kChunk ? t_end - t0 : kChunk);
         __syncthreads();  // previous chunk finished with every buffer
+
+        // ---- prologue: L2 norms of the q and k rows (one warp per row) ----
+        if constexpr (kPre) {
+            const int wp = tid >> 5, ln = tid & 31;
+            for (int r = wp; r < kChunk; r += kThreads / 32) {
+                float sq = 0.f, sk = 0.f;
+                if ((pre & GDR2_PROLOGUE_QK_L2NORM) && r < L) {
+                    for (int c = ln; c < DK; c += 32) {
+                        const int64_t i = ((t0 + r) * H + h) * DK + c;
+                        const float qv = to_f32(q[i]), kv = to_f32(k[i]);
+                        sq = fmaf(qv, qv, sq);
+                        sk = fmaf(kv, kv, sk);
+                    }
+                    for (int m = 16; m >= 1; m >>= 1) {
+                        sq += __shfl_xor_sync(0xffffffffu, sq, m);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, m);
+                    }
+                }
+                if (ln == 0) {
+                    const bool nrm = (pre & GDR2_PROLOGUE_QK_L2NORM) != 0;
+                    sm.qinv[r] = nrm ? rsqrtf(sq + 1e-6f) : 1.f;
+                    sm.kinv[r] = nrm ? rsqrtf(sk + 1e-6f) : 1.f;
+                }
+            }
+        }
+        if constexpr (kPre) __syncthreads();
 
         // ---- cumulative log-decay and decay-absorbed factors -------------
         if (tid < DK) {
@@ -93,7 +123,8 @@ chunk_simt_kernel(ChunkArgs args)
             float acc = 0.f;
 #pragma unroll
             for (int r = 0; r < kChunk; ++r) {
-                const float x = r < L ? la[((t0 + r) * H + h) * DK + c] : 0.f;
+                float x = r < L ? la[((t0 + r) * H + h) * DK + c] : 0.f;
+                if ((pre & GDR2_PROLOGUE_DECAY_SOFTPLUS) && r < L) x = pre_neg_softplus(x);
                 acc += x;
                 g[r] = acc;
             }
@@ -107,7 +138,12 @@ chunk_simt_kernel(ChunkArgs args)
                     const int64_t i = ((t0 + r) * H + h) * DK + c;
                     qv = to_f32(q[i]);
                     kv = to_f32(k[i]);
+                    if constexpr (kPre) {
+                        qv *= sm.qinv[r];
+                        kv *= sm.kinv[r];
+                    }
                     bv = to_f32(b[i]);
+                    if (pre & GDR2_PROLOGUE_GATE_SIGMOID) bv = pre_sigmoid(bv);
                 }
                 const float up = expf(g[r] - gm), dn = expf(gm - g[r]);
                 sm.qm[c][r] = qv * up;
@@ -120,7 +156,9 @@ chunk_simt_kernel(ChunkArgs args)
             float zv = 0.f;
             if (r < L) {
                 const int64_t e = ((t0 + r) * H + h) * DV + j0 + j;
-                zv = to_f32(w[e]) * to_f32(v[e]);
+                float wv = to_f32(w[e]);
+                if (pre & GDR2_PROLOGUE_GATE_SIGMOID) wv = pre_sigmoid(wv);
+                zv = wv * to_f32(v[e]);
             }
             sm.z[r][j] = zv;
         }
@@ -243,7 +281,7 @@ template <typename Tin, int DK>
 cudaError_t launch_t(const ChunkArgs &a, cudaStream_t stream)
 {
     const size_t smem = sizeof(SimtSmem<DK>);
-    auto kern = chunk_simt_kernel<Tin, DK>;
+    auto kern = a.pre ? chunk_simt_kernel<Tin, DK, true> : chunk_simt_kernel<Tin, DK, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(a.dv / kDVT), (unsigned)a.H, (unsigned)a.num_seqs);

@@ -172,6 +172,7 @@ struct TcParams {
     int64_t seg_len;
     __nv_bfloat16 *psi;
     float *seg_s0, *seg_phi;
+    uint32_t pre;  // GDR2_PROLOGUE_* flags (activations applied on load)
 };
 
 // Bounded wait on a barrier of this CTA (CTA-scope acquire: the peer's
@@ -298,6 +299,10 @@ __device__ __forceinline__ void store_row_bf16_sw128(unsigned char *tile, uint32
 __device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory"); }
 __device__ __forceinline__ void setmaxnreg_inc152() { asm volatile("setmaxnreg.inc.sync.aligned.u32 152;" ::: "memory"); }
 
+// kPre: the fused prologue is compiled in (only the *_preact calls launch it;
+// the plain kernel carries none of its code, which matters for instruction
+// fetch).
+template <bool kPre>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_v,
@@ -587,7 +592,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
                 const uint2 wr = *reinterpret_cast<const uint2 *>(w_tile + off);
                 const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
-                const float2 w0 = bf2_to_f2(wr.x), w1 = bf2_to_f2(wr.y);
+                float2 w0 = bf2_to_f2(wr.x), w1 = bf2_to_f2(wr.y);
+                if (kPre && (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID)) {
+                    w0 = make_float2(pre_sigmoid(w0.x), pre_sigmoid(w0.y));
+                    w1 = make_float2(pre_sigmoid(w1.x), pre_sigmoid(w1.y));
+                }
                 const bool ok = r < L;
                 uint2 oz;
                 oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
@@ -949,7 +958,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * pw + i;
-                const float4 x = *reinterpret_cast<const float4 *>(la_s + r * 128 + 4 * g);
+                float4 x = *reinterpret_cast<const float4 *>(la_s + r * 128 + 4 * g);
+                if (kPre && (prm.pre & GDR2_PROLOGUE_DECAY_SOFTPLUS))
+                    x = make_float4(pre_neg_softplus(x.x), pre_neg_softplus(x.y), pre_neg_softplus(x.z),
+                                    pre_neg_softplus(x.w));
                 la[i] = r < L ? x : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             float4 bs = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -999,6 +1011,36 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     }
                 }
             }
+            // prologue: 1 / ||q_r||, 1 / ||k_r|| (a warp holds whole rows: lanes
+            // 0-15 key channels 0-63, lanes 16-31 channels 64-127)
+            float qs[8], ks[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qs[i] = ks[i] = 1.f;
+            if (kPre && (prm.pre & GDR2_PROLOGUE_QK_L2NORM)) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t off = sw128_offset(8 * pw + i, cbyte);
+                    const uint2 qr = *reinterpret_cast<const uint2 *>(q_tile + off);
+                    const uint2 kr = *reinterpret_cast<const uint2 *>(k_tile + off);
+                    const float2 q0 = bf2_to_f2(qr.x), q1 = bf2_to_f2(qr.y);
+                    const float2 k0 = bf2_to_f2(kr.x), k1 = bf2_to_f2(kr.y);
+                    qs[i] = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
+                    ks[i] = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        qs[i] += __shfl_xor_sync(0xffffffffu, qs[i], m);
+                        ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], m);
+                    }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    qs[i] = rsqrtf(qs[i] + 1e-6f);
+                    ks[i] = rsqrtf(ks[i] + 1e-6f);
+                }
+            }
+            const bool gate_sig = kPre && (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID) != 0;
             // factors, in place: b -> Em, q -> Qm, k -> Km
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -1007,9 +1049,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const uint2 qr = *reinterpret_cast<const uint2 *>(q_tile + off);
                 const uint2 kr = *reinterpret_cast<const uint2 *>(k_tile + off);
                 const uint2 br = *reinterpret_cast<const uint2 *>(e_tile + off);
-                const float2 q0 = bf2_to_f2(qr.x), q1 = bf2_to_f2(qr.y);
-                const float2 k0 = bf2_to_f2(kr.x), k1 = bf2_to_f2(kr.y);
-                const float2 b0 = bf2_to_f2(br.x), b1 = bf2_to_f2(br.y);
+                float2 q0 = bf2_to_f2(qr.x), q1 = bf2_to_f2(qr.y);
+                float2 k0 = bf2_to_f2(kr.x), k1 = bf2_to_f2(kr.y);
+                float2 b0 = bf2_to_f2(br.x), b1 = bf2_to_f2(br.y);
+                if constexpr (kPre) {
+                    q0.x *= qs[i]; q0.y *= qs[i]; q1.x *= qs[i]; q1.y *= qs[i];
+                    k0.x *= ks[i]; k0.y *= ks[i]; k1.x *= ks[i]; k1.y *= ks[i];
+                }
+                if (gate_sig) {
+                    b0 = make_float2(pre_sigmoid(b0.x), pre_sigmoid(b0.y));
+                    b1 = make_float2(pre_sigmoid(b1.x), pre_sigmoid(b1.y));
+                }
                 const float u0 = ex2_approx(la[i].x), u1 = ex2_approx(la[i].y);
                 const float u2 = ex2_approx(la[i].z), u3 = ex2_approx(la[i].w);
                 const float v0 = ex2_approx(-la[i].x), v1 = ex2_approx(-la[i].y);
@@ -1330,12 +1380,13 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.units = units;
     p.nseg = a.nseg;
     p.seg_len = a.seg_len;
+    p.pre = a.pre;
     unsigned char *ws = static_cast<unsigned char *>(a.seg_ws);
     p.psi = a.nseg > 1 ? reinterpret_cast<__nv_bfloat16 *>(ws + seg_psi_offset()) : nullptr;
     p.seg_s0 = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_state_offset(a.B, a.T, a.H)) : nullptr;
     p.seg_phi = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_phi_offset(a.B, a.T, a.H, a.nseg)) : nullptr;
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    auto kernel = a.pre ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * kPairs * clusters), 1, 1);
@@ -1349,7 +1400,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chunk_tc_kernel, mq, mk, mb, mv, mla, mw, p);
+    return cudaLaunchKernelEx(&cfg, kernel, mq, mk, mb, mv, mla, mw, p);
 }
 
 namespace {

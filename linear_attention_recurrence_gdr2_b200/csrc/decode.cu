@@ -21,12 +21,13 @@
 
 namespace gdr2 {
 
-template <typename Tin, int DK, int DV, int NWARPS>
+// kPre: the fused prologue is compiled in (the *_preact calls only).
+template <typename Tin, int DK, int DV, int NWARPS, bool kPre>
 __global__ void __launch_bounds__(NWARPS * 32)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                    const Tin *__restrict__ v, const float *__restrict__ log_alpha,
                    const Tin *__restrict__ b, const Tin *__restrict__ w,
-                   float *__restrict__ state, Tin *__restrict__ o)
+                   float *__restrict__ state, Tin *__restrict__ o, uint32_t pre)
 {
     constexpr int VEC = DV / 32;          // value columns per lane
     constexpr int ROWS = DK / NWARPS;     // key rows per warp
@@ -40,17 +41,24 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     const int64_t head = blockIdx.x;   // n * H + h
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // (with the fused prologue: gates through a sigmoid, log_alpha through
+    // -softplus; q and k are normalised below where they are read)
     for (int c = threadIdx.x; c < DK; c += NWARPS * 32) {
         const int64_t i = head * DK + c;
         float kc = to_f32(k[i]);
-        s_alpha[c] = expf(log_alpha[i]);
-        s_e[c] = to_f32(b[i]) * kc;
+        float la = log_alpha[i], bc = to_f32(b[i]);
+        if (kPre && (pre & GDR2_PROLOGUE_DECAY_SOFTPLUS)) la = pre_neg_softplus(la);
+        if (kPre && (pre & GDR2_PROLOGUE_GATE_SIGMOID)) bc = pre_sigmoid(bc);
+        s_alpha[c] = expf(la);
+        s_e[c] = bc * kc;
         s_q[c] = to_f32(q[i]);
         s_k[c] = kc;
     }
     for (int j = threadIdx.x; j < DV; j += NWARPS * 32) {
         const int64_t i = head * DV + j;
-        s_z[j] = to_f32(w[i]) * to_f32(v[i]);
+        float wj = to_f32(w[i]);
+        if (kPre && (pre & GDR2_PROLOGUE_GATE_SIGMOID)) wj = pre_sigmoid(wj);
+        s_z[j] = wj * to_f32(v[i]);
     }
 
     // Issue every state load of this thread before the first use.
@@ -63,13 +71,30 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
     __syncthreads();
 
+    // prologue: 1 / ||q||, 1 / ||k|| (every warp reduces the shared copies itself)
+    float iq = 1.f, ik = 1.f;
+    if (kPre && (pre & GDR2_PROLOGUE_QK_L2NORM)) {
+        float sq = 0.f, sk = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+            sq = fmaf(s_q[c], s_q[c], sq);
+            sk = fmaf(s_k[c], s_k[c], sk);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        }
+        iq = rsqrtf(sq + 1e-6f);
+        ik = rsqrtf(sk + 1e-6f);
+    }
+
     float r[VEC], p[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) r[j] = p[j] = 0.f;
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
         const int c = warp + i * NWARPS;
-        const float a = s_alpha[c], e = s_e[c], qc = s_q[c];
+        const float a = s_alpha[c], e = kPre ? s_e[c] * ik : s_e[c], qc = kPre ? s_q[c] * iq : s_q[c];
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
             x[i][j] *= a;
@@ -87,6 +112,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     for (int c = lane; c < DK; c += 32) kq = fmaf(s_k[c], s_q[c], kq);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    if constexpr (kPre) kq *= ik * iq;
     __syncthreads();
 
     float u[VEC];
@@ -104,7 +130,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
         const int c = warp + i * NWARPS;
-        const float kc = s_k[c];
+        const float kc = kPre ? s_k[c] * ik : s_k[c];
         float *dst = S + (int64_t)c * DV + lane * VEC;
         float y[VEC];
 #pragma unroll
@@ -128,9 +154,10 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream)
     constexpr int NWARPS = 8;
     const int64_t heads = a.N * a.H;
     if (heads == 0) return cudaSuccess;
-    decode_step_kernel<Tin, D, D, NWARPS><<<(unsigned)heads, NWARPS * 32, 0, stream>>>(
+    auto kern = a.pre ? decode_step_kernel<Tin, D, D, NWARPS, true> : decode_step_kernel<Tin, D, D, NWARPS, false>;
+    kern<<<(unsigned)heads, NWARPS * 32, 0, stream>>>(
         (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, a.log_alpha,
-        (const Tin *)a.b, (const Tin *)a.w, a.state, (Tin *)a.o);
+        (const Tin *)a.b, (const Tin *)a.w, a.state, (Tin *)a.o, a.pre);
     return cudaGetLastError();
 }
 

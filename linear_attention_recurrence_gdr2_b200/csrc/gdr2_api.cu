@@ -8,7 +8,9 @@
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
+constexpr uint32_t kPrologueMask =
+    GDR2_PROLOGUE_QK_L2NORM | GDR2_PROLOGUE_GATE_SIGMOID | GDR2_PROLOGUE_DECAY_SOFTPLUS;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -81,6 +83,18 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
                            void *o, float *final_state, void *workspace,
                            size_t workspace_bytes, void *stream)
 {
+    return gdr2_chunk_fwd_preact(q, k, v, log_alpha, b, w, init_state, cu_seqlens, B, T, H, d_k, d_v,
+                                 num_seqs, dtype, o, final_state, workspace, workspace_bytes, 0u, stream);
+}
+
+gdr2_status gdr2_chunk_fwd_preact(const void *q, const void *k, const void *v, const float *log_alpha,
+                                  const void *b, const void *w, const float *init_state,
+                                  const int32_t *cu_seqlens, int64_t B, int64_t T, int64_t H,
+                                  int64_t d_k, int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                                  void *o, float *final_state, void *workspace,
+                                  size_t workspace_bytes, uint32_t prologue, void *stream)
+{
+    if (prologue & ~kPrologueMask) return GDR2_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
     if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
     gdr2_status st = check_dims(d_k, d_v);
@@ -126,6 +140,7 @@ gdr2_status gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     a.nseg = plan.nseg;
     a.seg_len = plan.seg_len;
     a.seg_ws = plan.nseg > 1 ? workspace : nullptr;
+    a.pre = prologue;
     cudaError_t e = cudaSuccess;
     if (cu_seqlens && num_seqs > 1) {
         a.order = static_cast<const int32_t *>(workspace);
@@ -147,6 +162,16 @@ gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
                                 float *state, int64_t N, int64_t H, int64_t d_k, int64_t d_v,
                                 gdr2_dtype dtype, void *o, void *stream)
 {
+    return gdr2_recurrent_step_preact(q, k, v, log_alpha, b, w, state, N, H, d_k, d_v, dtype, o, 0u,
+                                      stream);
+}
+
+gdr2_status gdr2_recurrent_step_preact(const void *q, const void *k, const void *v,
+                                       const float *log_alpha, const void *b, const void *w,
+                                       float *state, int64_t N, int64_t H, int64_t d_k, int64_t d_v,
+                                       gdr2_dtype dtype, void *o, uint32_t prologue, void *stream)
+{
+    if (prologue & ~kPrologueMask) return GDR2_ERR_INVALID_ARG;
     if (N < 0 || H <= 0) return GDR2_ERR_INVALID_ARG;
     if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
     gdr2_status st = check_dims(d_k, d_v);
@@ -164,6 +189,7 @@ gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,
     a.o = o;
     a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
     a.bf16 = dtype == GDR2_BF16;
+    a.pre = prologue;
     cudaError_t e = gdr2::launch_decode(a, (cudaStream_t)stream);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }

@@ -20,6 +20,7 @@ struct DecodeArgs {
     void *o;
     int64_t N, H, dk, dv;
     bool bf16;
+    uint32_t pre = 0;          // GDR2_PROLOGUE_* flags applied on load
 };
 
 struct ChunkArgs {
@@ -38,7 +39,12 @@ struct ChunkArgs {
     int nseg = 1;
     int64_t seg_len = 0;
     void *seg_ws = nullptr;
+    uint32_t pre = 0;          // GDR2_PROLOGUE_* flags applied on load
 };
+
+// The fused prologue's element-wise activations (fp32).
+__device__ __forceinline__ float pre_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float pre_neg_softplus(float x) { return x > 20.f ? -x : -log1pf(expf(x)); }
 
 // Segment plan of the tensor-core chunk forward: how many segments each
 // sequence of a fixed-length batch is split into (1 = none), and the scratch

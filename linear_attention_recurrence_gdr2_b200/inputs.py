@@ -186,3 +186,27 @@ def decode_batch(seed: int = 0, steps: int = 64, N: int = 256) -> DecodeInputs:
     """N=256 sequences x H=16 heads, d=128, fp32 state 0.01 * N(0,1),
     64 consecutive bf16 decode steps."""
     return make_decode_inputs(N, 16, 128, 128, steps, BF16, seed)
+
+
+def preact_inputs(B: int, T: int, H: int, d: int, dtype: str = BF16, seed: int = 0,
+                  init_std: Optional[float] = None, decay_shift: float = -2.5) -> Inputs:
+    """Pre-activation inputs for the fused prologue (gdr2_chunk_fwd_preact):
+    q, k ~ 2 N(0,1) (not normalised), v ~ N(0,1), b, w ~ 2 N(0,1) (before the
+    sigmoid), log_alpha ~ N(decay_shift, 1) (before -softplus: about -0.1 per
+    token for the default shift). Same rounding and draw order as make_inputs."""
+    rng = np.random.default_rng(seed)
+    sk, sv = (B, T, H, d), (B, T, H, d)
+    q = 2.0 * rng.standard_normal(sk, dtype=np.float32)
+    k = 2.0 * rng.standard_normal(sk, dtype=np.float32)
+    v = rng.standard_normal(sv, dtype=np.float32)
+    la = (rng.standard_normal(sk, dtype=np.float32) + np.float32(decay_shift)).astype(np.float32)
+    b = 2.0 * rng.standard_normal(sk, dtype=np.float32)
+    w = 2.0 * rng.standard_normal(sv, dtype=np.float32)
+    if dtype == BF16:
+        q, k, v, b, w = (round_to_bf16(x) for x in (q, k, v, b, w))
+    elif dtype != FP32:
+        raise ValueError(f"unknown dtype {dtype!r}")
+    s0 = None
+    if init_std is not None:
+        s0 = (rng.standard_normal((B, H, d, d), dtype=np.float32) * np.float32(init_std)).astype(np.float32)
+    return Inputs(q, k, v, la, b, w, s0, None, dtype, {"preact": True})

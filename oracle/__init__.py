@@ -11,7 +11,8 @@ enter the oracle with exactly the values the GPU sees.
 
 Pinned by: tests/test_oracle_pins.py (KDA and Gated DeltaNet reductions,
 exact recall, b=0 closed form, brute-force transition products, the
-fast-weight argmin identity, state passing, varlen splitting, linearity).
+fast-weight argmin identity, state passing, varlen splitting, linearity; the
+prologue against scipy's logistic function, numpy's logaddexp and norm).
 """
 from __future__ import annotations
 
@@ -132,3 +133,34 @@ def step(q, k, v, log_alpha, b, w, state, num_threads: int = 0):
     if rc != 0:
         raise ValueError(f"oracle step rejected its arguments (code {rc})")
     return o, S
+
+
+# Fused-prologue flags (the same bit values as GDR2_PROLOGUE_* in gdr2.h).
+PROLOGUE_QK_L2NORM = 1
+PROLOGUE_GATE_SIGMOID = 2
+PROLOGUE_DECAY_SOFTPLUS = 4
+
+
+def prologue(q, k, log_alpha, b, w, flags: int):
+    """The element-wise ends of the Gated DeltaNet-2 block's input branches, in
+    fp64 ("Block design and hybrid model", ainews.random.gg article: q and k
+    are L2-normalised, the erase and write gates are sigmoid projections; the
+    decay branch's activation is not printed, -softplus is the reading taken).
+
+    Per token and head, according to ``flags``:
+      PROLOGUE_QK_L2NORM:      q, k <- x / sqrt(sum_c x_c^2 + 1e-6)
+      PROLOGUE_GATE_SIGMOID:   b, w <- 1 / (1 + exp(-x))
+      PROLOGUE_DECAY_SOFTPLUS: log_alpha <- -log(1 + exp(x))
+    Returns (q, k, log_alpha, b, w) as float64 arrays.
+    """
+    q, k, la, b, w = (np.array(x, dtype=np.float64) for x in (q, k, log_alpha, b, w))
+    if flags & PROLOGUE_QK_L2NORM:
+        q = q / np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + 1e-6)
+        k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + 1e-6)
+    if flags & PROLOGUE_GATE_SIGMOID:
+        b = 1.0 / (1.0 + np.exp(-b))
+        w = 1.0 / (1.0 + np.exp(-w))
+    if flags & PROLOGUE_DECAY_SOFTPLUS:
+        # log(1 + e^x) = max(x, 0) + log(1 + e^{-|x|})  (no overflow)
+        la = -(np.maximum(la, 0.0) + np.log1p(np.exp(-np.abs(la))))
+    return q, k, la, b, w

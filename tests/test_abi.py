@@ -139,3 +139,15 @@ def test_empty_problems_return_ok_without_launch():
     assert _chunk(B=0, N=0, q=None, o=None) == OK
     assert _chunk(B=1, T=0, N=0, cu=FAKE) == OK
     assert _step(N=0, q=None, s=None) == OK
+
+
+def test_prologue_flags_validated():
+    """The *_preact entry points reject unknown prologue bits before anything else."""
+    L = gdr2.lib()
+    assert L.gdr2_chunk_fwd_preact(*([None] * 8), 1, 64, 1, 64, 64, 1, 0, None, None, None, 0, 8,
+                                   None) == INVALID
+    assert L.gdr2_recurrent_step_preact(*([None] * 7), 1, 1, 64, 64, 0, None, 8, None) == INVALID
+    # known bits pass the flag check and reach the usual validation (null pointers)
+    assert L.gdr2_chunk_fwd_preact(*([None] * 8), 1, 64, 1, 64, 64, 1, 0, None, None, None, 0, 7,
+                                   None) == INVALID
+    assert gdr2.GDR2_PROLOGUE_ALL == 7

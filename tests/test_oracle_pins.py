@@ -169,3 +169,32 @@ def test_segment_split_identity():
             s_start = np.einsum("nhik,nhkj->nhij", phi, s_start) + s_a
     assert np.max(np.abs(o - o_ref)) < 1e-12 * max(1.0, np.max(np.abs(o_ref)))
     assert np.max(np.abs(s_start - s_ref)) < 1e-12 * max(1.0, np.max(np.abs(s_ref)))
+
+
+def test_prologue_against_library_routines():
+    """The fused prologue's activations equal library routines: the logistic
+    function (scipy.special.expit), softplus (numpy.logaddexp(0, x)) and the
+    Euclidean norm (numpy.linalg.norm); no flag leaves the inputs unchanged;
+    each flag touches only its own tensors."""
+    from scipy.special import expit
+    rng = np.random.default_rng(5)
+    shp = (2, 7, 3, 16)
+    q, k, la, b, w = (rng.standard_normal(shp) * 3 for _ in range(5))
+    la[0, 0, 0, :4] = [-50.0, 50.0, 0.0, 700.0]   # extremes of softplus
+    same = oracle.prologue(q, k, la, b, w, 0)
+    for x, y in zip(same, (q, k, la, b, w)):
+        assert np.array_equal(x, y)
+    qn, kn, la2, bs, ws = oracle.prologue(q, k, la, b, w, 7)
+    eps = 1e-6
+    np.testing.assert_allclose(qn, q / np.sqrt(np.linalg.norm(q, axis=-1, keepdims=True) ** 2 + eps), rtol=1e-14)
+    np.testing.assert_allclose(kn, k / np.sqrt(np.linalg.norm(k, axis=-1, keepdims=True) ** 2 + eps), rtol=1e-14)
+    np.testing.assert_allclose(np.linalg.norm(qn, axis=-1), 1.0, rtol=1e-6)  # unit rows
+    np.testing.assert_allclose(bs, expit(b), rtol=1e-14)
+    np.testing.assert_allclose(ws, expit(w), rtol=1e-14)
+    np.testing.assert_allclose(la2, -np.logaddexp(0.0, la), rtol=1e-14)
+    assert np.all(la2 <= 0) and np.isfinite(la2).all()
+    # one flag at a time
+    q1, k1, la1, b1, w1 = oracle.prologue(q, k, la, b, w, oracle.PROLOGUE_GATE_SIGMOID)
+    assert np.array_equal(q1, q) and np.array_equal(k1, k) and np.array_equal(la1, la)
+    q1, k1, la1, b1, w1 = oracle.prologue(q, k, la, b, w, oracle.PROLOGUE_DECAY_SOFTPLUS)
+    assert np.array_equal(b1, b) and np.array_equal(w1, w) and np.array_equal(q1, q)

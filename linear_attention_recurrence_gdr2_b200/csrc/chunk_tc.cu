@@ -1,6 +1,6 @@
 // Chunkwise forward of Gated Delta Rule-2 for bf16 inputs, d_k = d_v = 128,
-// on the sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA), one
-// cluster of two CTAs per (sequence, head).
+// on the sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA), two
+// CTAs per (sequence, head) (a main and a helper; two such pairs per cluster).
 //
 // Chunk form (C = 64; "Chunkwise training and gate-aware backward" section
 // of the ainews.random.gg article on Gated DeltaNet-2). Per chunk with entry
@@ -19,17 +19,17 @@
 //
 // Work split. Only the state chain is serial across chunks; everything that
 // depends on one chunk's inputs alone runs ahead of it on a second SM:
-//   helper CTA (cluster rank 1), per chunk:
+//   helper CTA (cluster ranks 2, 3), per chunk:
 //     decay sums and factors Qm, Km, Em (in place over the q, k, b tiles),
 //     [A^T | P^T] = Km [Em; Qm]^T       M=64  N=128 K=128 (tcgen05),
 //     T = (I + A)^{-1} (tf32 mma.sync doubling) as bf16,
 //     and bulk copies of Em, Qm, Km, P^T, T and the half sums into the main
 //     CTA's shared memory (distributed shared memory inside the cluster);
-//   main CTA (cluster rank 0), per chunk:
-//     Z = w . v; W = T Em (two M=64 halves); U0^T = Z^T T^T;
+//   main CTA (cluster ranks 0, 1), per chunk:
+//     Z = w . v; -W = -(T Em) (two M=64 halves); U0^T = Z^T T^T;
 //     [U^T | O^T]  += Sm^T [-W; Qm]^T   M=128 N=128 K=128, A in TMEM
 //     [O^T | M^T]  += U^T [P^T | Km]    M=128 N=192 K=64,  A in TMEM
-//     and the epilogue (U^T to bf16, o stores, state scaling, final state).
+//     and the epilogue (U^T to bf16, o staging, state scaling, final state).
 // Everything is computed transposed so that the value dimension (128) sits
 // on the MMA's M axis and on the 128 TMEM lanes. The fp32 state lives in the
 // main CTA's TMEM (as M = Diag(e^{g_31}) S plus the chunk's update); once per
@@ -40,13 +40,15 @@
 // helper's copies complete on the main CTA's barriers.
 //
 // Warp roles (16 warps per CTA; the first warpgroup gives registers away):
-//   main:   0 v TMA producer, w L2 prefetch, slot-free relay
+//   main:   0 v and w TMA producer, slot-free relay
 //           1 tcgen05.mma issuer: W, U0      2 TMEM allocator, copy-landed relay
 //           3 tcgen05.mma issuer: state chain
-//           4..7 Z      8..11 -W from TMEM      12..15 epilogue
+//           4..7 Z      8..11 -W from TMEM, o stores      12..15 epilogue
 //   helper: 0 q, k, b TMA producer           1 tcgen05.mma issuer: [A^T | P^T]
-//           2 TMEM allocator                  4..11 decay factors, P^T
+//           2 TMEM allocator, factor sender   4..11 decay factors, P^T
 //           12..15 (I + A)^{-1}
+// With few long sequences one launch also runs the jobs of the segment-parallel
+// scan (segments.cu); a template flag compiles in the fused input prologue.
 // Every wait is bounded: after about a second without progress the CTA
 // records the site in the device error word, tells its peer to wind down,
 // drains its own TMA loads and MMAs, frees TMEM, and returns.

@@ -164,3 +164,66 @@ def prologue(q, k, log_alpha, b, w, flags: int):
         # log(1 + e^x) = max(x, 0) + log(1 + e^{-|x|})  (no overflow)
         la = -(np.maximum(la, 0.0) + np.log1p(np.exp(-np.abs(la))))
     return q, k, la, b, w
+
+
+def backward(q, k, v, log_alpha, b, w, init_state, d_o, d_final=None):
+    """Vector-Jacobian product of the token recurrence (fp64, plain numpy,
+    one token at a time in reverse, vectorised over (sequence, head) only).
+
+    The "Chunkwise training and gate-aware backward" section of the
+    ainews.random.gg article notes that with two different diagonal gates the
+    gate factors must appear inside the gradient's dot products; here they do
+    so by construction, by reverse-mode differentiation of the rule itself:
+        S'_t = Diag(alpha_t) S_{t-1},  e_t = b_t . k_t,  z_t = w_t . v_t,
+        r_t = S'_t^T e_t,  S_t = S'_t + k_t (z_t - r_t)^T,  o_t = S_t^T q_t.
+    With G = dL/dS_t (accumulated from the end, starting at d_final), each
+    step applies the chain rule to these five lines in reverse order (one line
+    of the body per term).
+    Fixed-length batches: tensors [B, T, H, d]; init_state [B, H, d_k, d_v] or
+    None; d_o like o; d_final [B, H, d_k, d_v] or None (zero).
+    Returns dq, dk, dv, dlog_alpha, db, dw, dinit_state (float64).
+    """
+    q, k, v, la, b, w, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, log_alpha, b, w, d_o))
+    B, T, H, dk_ = q.shape
+    dv_ = v.shape[-1]
+    S = (np.zeros((B, H, dk_, dv_)) if init_state is None
+         else np.array(init_state, dtype=np.float64, copy=True))
+    alpha = np.exp(la)
+    e = b * k
+    z = w * v
+    # forward, keeping every state S_{t-1} (input of step t)
+    prev = np.empty((T, B, H, dk_, dv_))
+    for t in range(T):
+        prev[t] = S
+        Sp = alpha[:, t, :, :, None] * S                       # S'_t = Diag(alpha_t) S_{t-1}
+        r = np.einsum("bhij,bhi->bhj", Sp, e[:, t])            # r_t = S'^T e_t
+        S = Sp + k[:, t, :, :, None] * (z[:, t] - r)[:, :, None, :]
+    G = np.zeros((B, H, dk_, dv_)) if d_final is None else np.array(d_final, dtype=np.float64, copy=True)
+    dq, dk, dv, dla, db, dw = (np.zeros_like(x) for x in (q, k, v, la, b, w))
+    for t in range(T - 1, -1, -1):
+        S_prev = prev[t]
+        Sp = alpha[:, t, :, :, None] * S_prev
+        r = np.einsum("bhij,bhi->bhj", Sp, e[:, t])
+        u = z[:, t] - r
+        S_t = Sp + k[:, t, :, :, None] * u[:, :, None, :]
+        # o_t = S_t^T q_t
+        G = G + q[:, t, :, :, None] * do[:, t, :, None, :]
+        dq[:, t] = np.einsum("bhij,bhj->bhi", S_t, do[:, t])
+        # S_t = S'_t + k_t u^T,  u = z_t - r_t
+        du = np.einsum("bhij,bhi->bhj", G, k[:, t])
+        dk_t = np.einsum("bhij,bhj->bhi", G, u)
+        dz = du
+        dr = -du
+        # r_t = S'^T e_t:  dS' += e dr^T,  de = S' dr
+        dSp = G + e[:, t, :, :, None] * dr[:, :, None, :]
+        de = np.einsum("bhij,bhj->bhi", Sp, dr)
+        # S'_t = Diag(alpha_t) S_{t-1}
+        dalpha = np.sum(dSp * S_prev, axis=-1)
+        G = alpha[:, t, :, :, None] * dSp
+        # e = b . k,  z = w . v,  alpha = exp(log_alpha)
+        db[:, t] = de * k[:, t]
+        dk[:, t] = dk_t + de * b[:, t]
+        dw[:, t] = dz * v[:, t]
+        dv[:, t] = dz * w[:, t]
+        dla[:, t] = dalpha * alpha[:, t]
+    return dq, dk, dv, dla, db, dw, G

@@ -183,6 +183,61 @@ gdr2_status gdr2_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                    void *o, float *final_state, void *stream);
 
 /*
+ * gdr2_chunk_bwd -- gate-aware backward (vector-Jacobian product) of the
+ * recurrence over whole sequences, for training.
+ *
+ * Given the forward's inputs and the cotangents dO of o and dS_T of the final
+ * states, returns the gradients of L = <dO, o> + <dS_T, S_T> with respect to
+ * q, k, v, log_alpha, b, w and the initial states. The "Chunkwise training
+ * and gate-aware backward" section of the ainews.random.gg article notes that
+ * with two different diagonal gates the gate factors enter the gradient's dot
+ * products; every gradient here is the chain rule of the token rule
+ *     S'_t = Diag(alpha_t) S_{t-1},  u_t = w_t.v_t - S'_t^T (b_t.k_t),
+ *     S_t = S'_t + k_t u_t^T,        o_t = S_t^T q_t,
+ * evaluated in fp32: a forward sweep and a reverse (cotangent) sweep along
+ * the tokens, each per value column, store per-token vectors and per-chunk
+ * (64 tokens) checkpoints in the workspace; a per-chunk pass then forms the
+ * key-side gradients row by row.
+ *
+ * Arguments (shapes as for gdr2_chunk_fwd; the same B, T, H, N, cu_seqlens)
+ *   q, k, v, log_alpha, b, w, init_state, cu_seqlens
+ *                the forward's inputs (init_state NULL = zero)
+ *   d_o          [B, T, H, d_v] in `dtype`: cotangent of o
+ *   d_final_state [N, H, d_k, d_v] fp32: cotangent of the final states, or
+ *                NULL for zero
+ *   dq, dk, db   [B, T, H, d_k] in `dtype` (outputs)
+ *   dv, dw       [B, T, H, d_v] in `dtype` (outputs)
+ *   d_log_alpha  [B, T, H, d_k] fp32 (output)
+ *   d_init_state [N, H, d_k, d_v] fp32 (output), or NULL to skip it; may
+ *                alias d_final_state
+ *   workspace, workspace_bytes
+ *                device scratch of at least gdr2_chunk_bwd_workspace_size()
+ *                bytes, 16-byte aligned (required whenever N > 0); contents
+ *                are overwritten
+ * Outputs may not alias inputs (except d_init_state / d_final_state). Inputs
+ * are the post-activation values (there is no prologue variant). Errors as
+ * for gdr2_chunk_fwd; GDR2_ERR_WORKSPACE if the workspace is missing or small.
+ */
+gdr2_status gdr2_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const void *b, const void *w,
+                           const float *init_state, const int32_t *cu_seqlens,
+                           const void *d_o, const float *d_final_state,
+                           int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                           int64_t num_seqs, gdr2_dtype dtype,
+                           void *dq, void *dk, void *dv, float *d_log_alpha,
+                           void *db, void *dw, float *d_init_state,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Scratch bytes gdr2_chunk_bwd needs (written to *bytes), a multiple of 256:
+ * with S = B*T/64 + N checkpoint slots (integer division), 2 * S*H*d_k*d_v*4
+ * bytes of fp32 checkpoints plus 2 * B*T*H*d_v*4 bytes of per-token fp32
+ * vectors. */
+gdr2_status gdr2_chunk_bwd_workspace_size(int64_t B, int64_t T, int64_t H,
+                                          int64_t d_k, int64_t d_v,
+                                          int64_t num_seqs, gdr2_dtype dtype,
+                                          size_t *bytes);
+
+/*
  * gdr2_recurrent_step -- one decode step for N independent sequences.
  *
  * For every sequence n and head h, with the state updated IN PLACE:

@@ -11,6 +11,8 @@ Entry points (same names as the C ABI):
   chunk_fwd(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None)
       -> (o, final_state)
   recurrent_step(q, k, v, log_alpha, b, w, state) -> o   (state in place)
+  chunk_bwd(q, k, v, log_alpha, b, w, d_o, init_state=None, d_final_state=None,
+            cu_seqlens=None) -> (dq, dk, dv, d_log_alpha, db, dw, d_init_state)
 """
 from __future__ import annotations
 
@@ -88,6 +90,14 @@ def lib() -> ctypes.CDLL:
             L.gdr2_recurrent_step_preact.argtypes = [
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                 _i64, _i64, _i64, _i64, ctypes.c_int, _vp, ctypes.c_uint32, _vp]
+            L.gdr2_chunk_bwd_workspace_size.restype = ctypes.c_int
+            L.gdr2_chunk_bwd_workspace_size.argtypes = [
+                _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+            L.gdr2_chunk_bwd.restype = ctypes.c_int
+            L.gdr2_chunk_bwd.argtypes = [
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             _lib = L
     return _lib
 
@@ -147,6 +157,65 @@ def workspace_size(B: int, T: int, H: int, d_k: int, d_v: int, num_seqs: int,
     if st != GDR2_OK:
         raise GDR2Error("gdr2_chunk_fwd_workspace_size", st)
     return int(out.value)
+
+
+def bwd_workspace_size(B: int, T: int, H: int, d_k: int, d_v: int, num_seqs: int,
+                       dtype_code: int) -> int:
+    out = ctypes.c_size_t(0)
+    st = lib().gdr2_chunk_bwd_workspace_size(B, T, H, d_k, d_v, num_seqs, dtype_code,
+                                             ctypes.byref(out))
+    if st != GDR2_OK:
+        raise GDR2Error("gdr2_chunk_bwd_workspace_size", st)
+    return int(out.value)
+
+
+def chunk_bwd(q, k, v, log_alpha, b, w, d_o, init_state=None, d_final_state=None,
+              cu_seqlens=None, *, output_d_init_state: bool = True, workspace=None,
+              stream=None):
+    """Gate-aware backward of Gated Delta Rule-2 (see gdr2_chunk_bwd in gdr2.h).
+
+    Same inputs as chunk_fwd plus d_o (cotangent of o, like o) and
+    d_final_state ([N, H, d_k, d_v] fp32 or None = zero). Returns
+    (dq, dk, dv, d_log_alpha, db, dw, d_init_state): the first six like their
+    inputs (d_log_alpha fp32), d_init_state [N, H, d_k, d_v] fp32 or None.
+    """
+    import torch
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("chunk_bwd needs CUDA tensors")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("k", k, dk), ("b", b, dk), ("v", v, dv), ("w", w, dv), ("d_o", d_o, dv)):
+        _check(t, name, (B, T, H, d), dt, dev)
+    _check(q, "q", (B, T, H, dk), dt, dev)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+        N = cu_seqlens.shape[0] - 1
+    else:
+        N = B
+    for name, t in (("init_state", init_state), ("d_final_state", d_final_state)):
+        if t is not None:
+            _check(t, name, (N, H, dk, dv), torch.float32, dev)
+    dq, dk_, db = (torch.empty((B, T, H, dk), dtype=dt, device=dev) for _ in range(3))
+    dv_, dw = (torch.empty((B, T, H, dv), dtype=dt, device=dev) for _ in range(2))
+    dla = torch.empty((B, T, H, dk), dtype=torch.float32, device=dev)
+    d_init = (torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+              if output_d_init_state else None)
+    need = bwd_workspace_size(B, T, H, dk, dv, N, code)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib().gdr2_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(init_state),
+        _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv, N, code,
+        _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(db), _ptr(dw), _ptr(d_init),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != GDR2_OK:
+        raise GDR2Error("gdr2_chunk_bwd", st)
+    return dq, dk_, dv_, dla, db, dw, d_init
 
 
 def chunk_fwd(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None, *,

@@ -1,0 +1,497 @@
+// Gate-aware backward of Gated Delta Rule-2: the vector-Jacobian product of
+//   S'_t = Diag(alpha_t) S_{t-1},  e_t = b_t . k_t,  z_t = w_t . v_t,
+//   u_t  = z_t - S'_t^T e_t,       S_t = S'_t + k_t u_t^T,  o_t = S_t^T q_t
+// for cotangents dO (per token) and dS_T (per sequence). The "Chunkwise
+// training and gate-aware backward" section of the ainews.random.gg article on
+// Gated DeltaNet-2 notes that with two different diagonal gates the gate
+// factors must sit inside the gradient's dot products; here every gradient is
+// the exact chain rule of the lines above, taken in fp32.
+//
+// Decomposition (three sweeps, two launches):
+//   A (forward, per value column j): the rule above only mixes key rows, so
+//     column j of S evolves on its own given alpha, e, k and z_{t,j}. Stores
+//     u_t and the state at every chunk start (checkpoints, fp32).
+//   B (reverse, per value column j): with H_t = G + q_t do_t^T,
+//     du_t = H_t^T k_t and G <- Diag(alpha_t)(H_t - e_t du_t^T), starting from
+//     dS_T, column j of G also evolves on its own. Stores du_t and G at every
+//     chunk end; writes dv = du . w, dw = du . v and dS_0 (the last G).
+//   C (per chunk and key row i): given u and du, row i of S (forward from the
+//     chunk-start checkpoint) and row i of H (reverse from the chunk-end one)
+//     evolve on their own, so every remaining gradient is a row-local dot
+//     product over value columns:
+//       dq_t = S_t do_t,  de_t = -S'_t du_t,  dkW_t = H_t u_t,
+//       dk_t = dkW_t + b_t . de_t,  db_t = k_t . de_t,
+//       dlog_alpha_t = sum_{s >= t in the chunk} (q.dq - k.dkW + e.de)_s
+//                      + rowsum(G_end . S_end).
+//     The last line replaces the per-token rowsum(dS'_t . S'_t): both
+//     recurrences telescope, so the decay gradient of token t is that of
+//     token t+1 plus the three per-token terms, and at a chunk end it equals
+//     the row-wise product of the incoming cotangent with the state there.
+//     Restarting it at every chunk end keeps its cancellation within 64 tokens.
+// A and B run in one launch (blockIdx.z picks the sweep); C follows on the
+// same stream. All arithmetic is fp32 on the CUDA cores.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdr2 {
+namespace {
+
+constexpr int kSub = 16;           // tokens staged per round of the column sweeps
+constexpr int kScanThreads = 256;  // 8 warps; a half-warp per pair of value columns
+constexpr int kTile = 32;          // value columns per column-sweep CTA
+constexpr int kRowThreads = 256;   // 4 lanes per key row in the per-chunk kernel
+
+struct BwdParams {
+    const void *q, *k, *v, *b, *w, *d_o;
+    const float *la, *init_state, *d_final;
+    const int32_t *cu;
+    void *dq, *dk, *dv, *db, *dw;
+    float *dla, *d_init;
+    float *ck, *gk, *U, *dU;   // workspace: checkpoints and per-token column vectors
+    int64_t T, H, N, tokens;
+};
+
+// Token range of sequence n (packed offsets are clamped to the token count).
+__device__ __forceinline__ void seq_bounds(const BwdParams &p, int64_t n, int64_t &start, int64_t &len)
+{
+    if (p.cu) {
+        int64_t s = p.cu[n], e = p.cu[n + 1];
+        s = s < 0 ? 0 : (s > p.tokens ? p.tokens : s);
+        e = e < s ? s : (e > p.tokens ? p.tokens : e);
+        start = s;
+        len = e - s;
+    } else {
+        start = n * p.T;
+        len = p.T;
+    }
+}
+
+// First checkpoint slot of sequence n. start/64 + n grows by at least
+// ceil(len/64) from one sequence to the next, so the slots of different
+// sequences never overlap and all lie below tokens/64 + N.
+__device__ __forceinline__ int64_t slot_base(int64_t start, int64_t n) { return start / kChunk + n; }
+
+template <typename T>
+__device__ __forceinline__ void store2(T *p, float a, float b);
+template <>
+__device__ __forceinline__ void store2<float>(float *p, float a, float b) {
+    *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+}
+template <>
+__device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16 *p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
+}
+
+// Sweeps A (blockIdx.z == 0) and B (blockIdx.z == 1). CTA = (sequence, head,
+// tile of 32 value columns); lane l of warp w owns columns 32*tile + 4w +
+// 2*(l/16) + {0,1} and key rows (l % 16) + 16m, so the reductions over key rows
+// are four xor-shuffles inside a half-warp. Row inputs (alpha, e, k, q) for 16
+// tokens are staged in shared memory, the next 16 prefetched into registers
+// while the current ones are consumed.
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
+{
+    constexpr int ROWS = D / 16;
+    constexpr int PF = kSub * D / kScanThreads;           // staged row elements per thread
+    constexpr int PC = kSub * kTile / kScanThreads;       // staged column elements per thread
+    static_assert(PF * kScanThreads == kSub * D && PC * kScanThreads == kSub * kTile, "staging split");
+    __shared__ float s_al[kSub * D], s_e[kSub * D], s_k[kSub * D], s_q[kSub * D];
+    __shared__ float s_c[3][kSub * kTile];   // A: z | B: do, v, w
+
+    const int64_t n = blockIdx.x / p.H;
+    const int h = (int)(blockIdx.x % p.H);
+    const int tile = blockIdx.y;
+    const bool rev = blockIdx.z != 0;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rho = lane & 15;
+    const int jl = warp * 4 + (lane >> 4) * 2;   // first of this lane's two columns, in the tile
+    const int j = tile * kTile + jl;
+    const Tin *Q = static_cast<const Tin *>(p.q), *K = static_cast<const Tin *>(p.k);
+    const Tin *Bg = static_cast<const Tin *>(p.b), *V = static_cast<const Tin *>(p.v);
+    const Tin *Wg = static_cast<const Tin *>(p.w), *DO = static_cast<const Tin *>(p.d_o);
+
+    int64_t start, len;
+    seq_bounds(p, n, start, len);
+    const int64_t base = slot_base(start, n);
+    const int64_t nsub = (len + kSub - 1) / kSub;
+    const int64_t head_state = (n * p.H + h) * (int64_t)D * D;
+
+    // X: state columns (A) or cotangent columns (B), rows rho + 16m
+    float X0[ROWS], X1[ROWS];
+    const float *x_init = rev ? p.d_final : p.init_state;
+#pragma unroll
+    for (int m = 0; m < ROWS; ++m) {
+        if (x_init) {
+            const float2 v2 = *reinterpret_cast<const float2 *>(x_init + head_state + (int64_t)(rho + 16 * m) * D + j);
+            X0[m] = v2.x;
+            X1[m] = v2.y;
+        } else {
+            X0[m] = 0.f;
+            X1[m] = 0.f;
+        }
+    }
+
+    float pf_la[PF], pf_k[PF], pf_b[PF], pf_q[PF], pc0[PC], pc1[PC], pc2[PC];
+    auto prefetch = [&](int64_t sb) {
+        const int64_t t0 = sb * kSub;
+#pragma unroll
+        for (int x = 0; x < PF; ++x) {
+            const int idx = tid + x * kScanThreads;
+            const int tt = idx / D, i = idx % D;
+            pf_la[x] = 0.f; pf_k[x] = 0.f; pf_b[x] = 0.f; pf_q[x] = 0.f;
+            if (t0 + tt < len) {
+                const int64_t off = ((start + t0 + tt) * p.H + h) * D + i;
+                pf_la[x] = p.la[off];
+                pf_k[x] = to_f32(K[off]);
+                pf_b[x] = to_f32(Bg[off]);
+                if (rev) pf_q[x] = to_f32(Q[off]);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < PC; ++x) {
+            const int idx = tid + x * kScanThreads;
+            const int tt = idx / kTile, jj = idx % kTile;
+            pc0[x] = 0.f; pc1[x] = 0.f; pc2[x] = 0.f;
+            if (t0 + tt < len) {
+                const int64_t off = ((start + t0 + tt) * p.H + h) * D + tile * kTile + jj;
+                const float vv = to_f32(V[off]), ww = to_f32(Wg[off]);
+                if (rev) {
+                    pc0[x] = to_f32(DO[off]);
+                    pc1[x] = vv;
+                    pc2[x] = ww;
+                } else {
+                    pc0[x] = ww * vv;
+                }
+            }
+        }
+    };
+
+    if (nsub > 0) prefetch(rev ? nsub - 1 : 0);
+    for (int64_t it = 0; it < nsub; ++it) {
+        const int64_t sb = rev ? nsub - 1 - it : it;
+        __syncthreads();   // the previous round's shared reads are done
+#pragma unroll
+        for (int x = 0; x < PF; ++x) {
+            const int idx = tid + x * kScanThreads;   // = tt * D + i
+            s_al[idx] = expf(pf_la[x]);
+            s_e[idx] = pf_b[x] * pf_k[x];
+            s_k[idx] = pf_k[x];
+            s_q[idx] = pf_q[x];
+        }
+#pragma unroll
+        for (int x = 0; x < PC; ++x) {
+            const int idx = tid + x * kScanThreads;   // = tt * kTile + jj
+            s_c[0][idx] = pc0[x];
+            s_c[1][idx] = pc1[x];
+            s_c[2][idx] = pc2[x];
+        }
+        __syncthreads();
+        if (rev ? sb > 0 : sb + 1 < nsub) prefetch(rev ? sb - 1 : sb + 1);
+
+        const int L = (int)((len - sb * kSub) < kSub ? (len - sb * kSub) : kSub);
+        const int64_t chunk = sb / (kChunk / kSub);
+        const bool at_chunk_edge = rev ? (sb % (kChunk / kSub) == kChunk / kSub - 1 || sb == nsub - 1)
+                                       : (sb % (kChunk / kSub) == 0);
+        if (at_chunk_edge) {
+            // A: state at the chunk start; B: cotangent of the state at the chunk end
+            float *dst = (rev ? p.gk : p.ck) + ((base + chunk) * p.H + h) * (int64_t)D * D;
+#pragma unroll
+            for (int m = 0; m < ROWS; ++m)
+                *reinterpret_cast<float2 *>(dst + (int64_t)(rho + 16 * m) * D + j) = make_float2(X0[m], X1[m]);
+        }
+
+        if (!rev) {
+            for (int tt = 0; tt < L; ++tt) {
+                const int64_t tok = start + sb * kSub + tt;
+                float r0 = 0.f, r1 = 0.f, kk[ROWS];
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m) {
+                    const int i = tt * D + rho + 16 * m;
+                    const float a = s_al[i], e = s_e[i];
+                    kk[m] = s_k[i];
+                    X0[m] *= a;                       // S' = Diag(alpha) S
+                    X1[m] *= a;
+                    r0 = fmaf(X0[m], e, r0);          // r = S'^T e
+                    r1 = fmaf(X1[m], e, r1);
+                }
+#pragma unroll
+                for (int off = 8; off >= 1; off >>= 1) {
+                    r0 += __shfl_xor_sync(0xffffffffu, r0, off);
+                    r1 += __shfl_xor_sync(0xffffffffu, r1, off);
+                }
+                const float u0 = s_c[0][tt * kTile + jl] - r0, u1 = s_c[0][tt * kTile + jl + 1] - r1;
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m) {
+                    X0[m] = fmaf(kk[m], u0, X0[m]);   // S = S' + k u^T
+                    X1[m] = fmaf(kk[m], u1, X1[m]);
+                }
+                if (rho == 0)
+                    *reinterpret_cast<float2 *>(p.U + (tok * p.H + h) * D + j) = make_float2(u0, u1);
+            }
+        } else {
+            for (int tt = L - 1; tt >= 0; --tt) {
+                const int64_t tok = start + sb * kSub + tt;
+                const int c = tt * kTile + jl;
+                const float o0 = s_c[0][c], o1 = s_c[0][c + 1];
+                float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m) {
+                    const int i = tt * D + rho + 16 * m;
+                    const float qi = s_q[i], ki = s_k[i];
+                    X0[m] = fmaf(qi, o0, X0[m]);      // H = G + q do^T
+                    X1[m] = fmaf(qi, o1, X1[m]);
+                    d0 = fmaf(X0[m], ki, d0);         // du = H^T k
+                    d1 = fmaf(X1[m], ki, d1);
+                }
+#pragma unroll
+                for (int off = 8; off >= 1; off >>= 1) {
+                    d0 += __shfl_xor_sync(0xffffffffu, d0, off);
+                    d1 += __shfl_xor_sync(0xffffffffu, d1, off);
+                }
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m) {
+                    const int i = tt * D + rho + 16 * m;
+                    const float a = s_al[i], e = s_e[i];
+                    X0[m] = a * fmaf(-e, d0, X0[m]);  // G = Diag(alpha)(H - e du^T)
+                    X1[m] = a * fmaf(-e, d1, X1[m]);
+                }
+                if (rho == 0) {
+                    const int64_t off = (tok * p.H + h) * D + j;
+                    *reinterpret_cast<float2 *>(p.dU + off) = make_float2(d0, d1);
+                    store2(static_cast<Tin *>(p.dv) + off, d0 * s_c[2][c], d1 * s_c[2][c + 1]);  // du . w
+                    store2(static_cast<Tin *>(p.dw) + off, d0 * s_c[1][c], d1 * s_c[1][c + 1]);  // du . v
+                }
+            }
+        }
+    }
+    if (rev && p.d_init) {
+#pragma unroll
+        for (int m = 0; m < ROWS; ++m)
+            *reinterpret_cast<float2 *>(p.d_init + head_state + (int64_t)(rho + 16 * m) * D + j) =
+                make_float2(X0[m], X1[m]);
+    }
+}
+
+// Sweep C. CTA = (checkpoint slot, head); thread = (key rows rg + 64r, lane s
+// of 4), lane s holding value columns 4(s + 4g) .. +3. Row reductions over
+// value columns are two xor-shuffles inside each group of 4 lanes.
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
+{
+    constexpr int RPT = D / 64;   // key rows per thread
+    constexpr int NG = D / 16;    // float4 column groups per thread
+    __shared__ float s_g[kChunk][D];   // dkW of the chunk, then the per-token decay terms
+
+    const int64_t slot = blockIdx.x;
+    const int h = blockIdx.y;
+    // the sequence that owns this slot: the last n with slot_base(n) <= slot
+    int64_t lo = 0, hi = p.N - 1;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) >> 1;
+        int64_t s_mid, l_mid;
+        seq_bounds(p, mid, s_mid, l_mid);
+        if (slot_base(s_mid, mid) <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    int64_t start, len;
+    seq_bounds(p, lo, start, len);
+    const int64_t c = slot - slot_base(start, lo);
+    if (c < 0 || c * kChunk >= len) return;   // an unused slot
+    const int64_t t0 = start + c * kChunk;
+    const int L = (int)((len - c * kChunk) < kChunk ? (len - c * kChunk) : kChunk);
+
+    const int tid = threadIdx.x, s = tid & 3, rg = tid >> 2;
+    const Tin *Q = static_cast<const Tin *>(p.q), *K = static_cast<const Tin *>(p.k);
+    const Tin *Bg = static_cast<const Tin *>(p.b), *DO = static_cast<const Tin *>(p.d_o);
+    const int64_t slot_off = (slot * p.H + h) * (int64_t)D * D;
+
+    float X[RPT][NG][4];
+    // pass R: H from the chunk-end cotangent, tokens in reverse
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(p.gk + slot_off + (int64_t)(rg + 64 * r) * D + 4 * (s + 4 * g));
+            X[r][g][0] = v4.x; X[r][g][1] = v4.y; X[r][g][2] = v4.z; X[r][g][3] = v4.w;
+        }
+    for (int tt = L - 1; tt >= 0; --tt) {
+        const int64_t row0 = ((t0 + tt) * p.H + h) * D;
+        float qr[RPT], ar[RPT], er[RPT], acc[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int64_t o = row0 + rg + 64 * r;
+            qr[r] = to_f32(Q[o]);
+            ar[r] = expf(p.la[o]);
+            er[r] = to_f32(Bg[o]) * to_f32(K[o]);
+            acc[r] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const int col = 4 * (s + 4 * g);
+            float o4[4];
+            load_vec<Tin, 4>(DO + row0 + col, o4);
+            const float4 u4 = *reinterpret_cast<const float4 *>(p.U + row0 + col);
+            const float4 d4 = *reinterpret_cast<const float4 *>(p.dU + row0 + col);
+            const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    float hv = fmaf(qr[r], o4[x], X[r][g][x]);   // H = G + q do^T
+                    acc[r] = fmaf(hv, uu[x], acc[r]);            // dkW = H u
+                    X[r][g][x] = ar[r] * fmaf(-er[r], dd[x], hv); // G = alpha (H - e du^T)
+                }
+        }
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+            acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 2);
+            if (s == 0) s_g[tt][rg + 64 * r] = acc[r];
+        }
+    }
+    __syncwarp();
+
+    // pass F: S from the chunk-start state, tokens in order
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(p.ck + slot_off + (int64_t)(rg + 64 * r) * D + 4 * (s + 4 * g));
+            X[r][g][0] = v4.x; X[r][g][1] = v4.y; X[r][g][2] = v4.z; X[r][g][3] = v4.w;
+        }
+    Tin *DQ = static_cast<Tin *>(p.dq), *DK = static_cast<Tin *>(p.dk), *DB = static_cast<Tin *>(p.db);
+    for (int tt = 0; tt < L; ++tt) {
+        const int64_t row0 = ((t0 + tt) * p.H + h) * D;
+        float qr[RPT], kr[RPT], br[RPT], ar[RPT], de[RPT], dq[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int64_t o = row0 + rg + 64 * r;
+            qr[r] = to_f32(Q[o]);
+            kr[r] = to_f32(K[o]);
+            br[r] = to_f32(Bg[o]);
+            ar[r] = expf(p.la[o]);
+            de[r] = 0.f;
+            dq[r] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const int col = 4 * (s + 4 * g);
+            float o4[4];
+            load_vec<Tin, 4>(DO + row0 + col, o4);
+            const float4 u4 = *reinterpret_cast<const float4 *>(p.U + row0 + col);
+            const float4 d4 = *reinterpret_cast<const float4 *>(p.dU + row0 + col);
+            const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float sp = ar[r] * X[r][g][x];          // S' = alpha S
+                    de[r] = fmaf(sp, dd[x], de[r]);               // S' du
+                    X[r][g][x] = fmaf(kr[r], uu[x], sp);          // S = S' + k u^T
+                    dq[r] = fmaf(X[r][g][x], o4[x], dq[r]);       // S do
+                }
+        }
+        float dkv[RPT], dbv[RPT], dgv[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            de[r] += __shfl_xor_sync(0xffffffffu, de[r], 1);
+            de[r] += __shfl_xor_sync(0xffffffffu, de[r], 2);
+            dq[r] += __shfl_xor_sync(0xffffffffu, dq[r], 1);
+            dq[r] += __shfl_xor_sync(0xffffffffu, dq[r], 2);
+            const float dev = -de[r];
+            const float dkw = s_g[tt][rg + 64 * r];
+            dkv[r] = fmaf(br[r], dev, dkw);                       // dk = dkW + b . de
+            dbv[r] = kr[r] * dev;                                 // db = k . de
+            dgv[r] = qr[r] * dq[r] - kr[r] * dkw + br[r] * kr[r] * dev;  // q.dq - k.dkW + e.de
+        }
+        __syncwarp();   // every lane has read s_g[tt] before lane 3 overwrites it
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int64_t o = row0 + rg + 64 * r;
+            if (s == 0) DQ[o] = from_f32<Tin>(dq[r]);
+            else if (s == 1) DK[o] = from_f32<Tin>(dkv[r]);
+            else if (s == 2) DB[o] = from_f32<Tin>(dbv[r]);
+            else s_g[tt][rg + 64 * r] = dgv[r];
+        }
+    }
+    // rowsum(G_end . S_end), then the reverse cumulative sum of the decay terms
+    float bt[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        bt[r] = 0.f;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(p.gk + slot_off + (int64_t)(rg + 64 * r) * D + 4 * (s + 4 * g));
+            bt[r] = fmaf(v4.x, X[r][g][0], bt[r]);
+            bt[r] = fmaf(v4.y, X[r][g][1], bt[r]);
+            bt[r] = fmaf(v4.z, X[r][g][2], bt[r]);
+            bt[r] = fmaf(v4.w, X[r][g][3], bt[r]);
+        }
+        bt[r] += __shfl_xor_sync(0xffffffffu, bt[r], 1);
+        bt[r] += __shfl_xor_sync(0xffffffffu, bt[r], 2);
+    }
+    __syncwarp();   // lane 3's decay terms are visible to the lanes that sum them
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        if (s == r) {
+            float acc = bt[r];
+            for (int tt = L - 1; tt >= 0; --tt) {
+                acc += s_g[tt][rg + 64 * r];
+                p.dla[((t0 + tt) * p.H + h) * D + rg + 64 * r] = acc;
+            }
+        }
+    }
+}
+
+template <typename Tin, int D>
+cudaError_t launch_typed(const BwdParams &p, int64_t slots, cudaStream_t stream)
+{
+    if (p.N * p.H > 0) {
+        dim3 grid((unsigned)(p.N * p.H), D / kTile, 2);
+        bwd_scan_kernel<Tin, D><<<grid, kScanThreads, 0, stream>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (p.tokens > 0) {
+        dim3 grid((unsigned)slots, (unsigned)p.H);
+        bwd_rows_kernel<Tin, D><<<grid, kRowThreads, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+int64_t bwd_slots(int64_t tokens, int64_t num_seqs) { return tokens / kChunk + num_seqs; }
+
+size_t bwd_workspace_bytes(int64_t tokens, int64_t H, int64_t d, int64_t num_seqs)
+{
+    const size_t states = (size_t)bwd_slots(tokens, num_seqs) * H * d * d * sizeof(float);
+    const size_t vecs = (size_t)tokens * H * d * sizeof(float);
+    const size_t bytes = 2 * states + 2 * vecs;
+    return (bytes + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)
+{
+    BwdParams p;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.b = a.b; p.w = a.w; p.d_o = a.d_o;
+    p.la = a.log_alpha; p.init_state = a.init_state; p.d_final = a.d_final;
+    p.cu = a.cu_seqlens;
+    p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.db = a.db; p.dw = a.dw;
+    p.dla = a.d_log_alpha; p.d_init = a.d_init_state;
+    p.T = a.T; p.H = a.H; p.N = a.num_seqs; p.tokens = a.B * a.T;
+    const int64_t slots = bwd_slots(p.tokens, p.N);
+    const size_t states = (size_t)slots * a.H * a.d * a.d;
+    float *ws = static_cast<float *>(a.workspace);
+    p.ck = ws;
+    p.gk = ws + states;
+    p.U = ws + 2 * states;
+    p.dU = p.U + (size_t)p.tokens * a.H * a.d;
+    if (a.bf16)
+        return a.d == 128 ? launch_typed<__nv_bfloat16, 128>(p, slots, stream)
+                          : launch_typed<__nv_bfloat16, 64>(p, slots, stream);
+    return a.d == 128 ? launch_typed<float, 128>(p, slots, stream) : launch_typed<float, 64>(p, slots, stream);
+}
+
+}  // namespace gdr2

@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kVersion = 200;  // 0.2.0
+constexpr int kVersion = 300;  // 0.3.0
 constexpr uint32_t kPrologueMask =
     GDR2_PROLOGUE_QK_L2NORM | GDR2_PROLOGUE_GATE_SIGMOID | GDR2_PROLOGUE_DECAY_SOFTPLUS;
 
@@ -155,6 +155,68 @@ gdr2_status gdr2_chunk_fwd_preact(const void *q, const void *k, const void *v, c
         e = gdr2::launch_chunk_simt(a, (cudaStream_t)stream);
     }
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+gdr2_status gdr2_chunk_bwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t d_k,
+                                          int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                                          size_t *bytes)
+{
+    if (!bytes) return GDR2_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    *bytes = gdr2::bwd_workspace_bytes(B * T, H, d_k, num_seqs);
+    return GDR2_OK;
+}
+
+gdr2_status gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *init_state,
+                           const int32_t *cu_seqlens, const void *d_o, const float *d_final_state,
+                           int64_t B, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                           int64_t num_seqs, gdr2_dtype dtype, void *dq, void *dk, void *dv,
+                           float *d_log_alpha, void *db, void *dw, float *d_init_state,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    if (cu_seqlens) {
+        if (B != 1) return GDR2_ERR_INVALID_ARG;
+    } else if (num_seqs != B) {
+        return GDR2_ERR_INVALID_ARG;
+    }
+    if (H > 65535 || num_seqs * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;
+    const int64_t tokens = B * T;
+    if (tokens > 0) {
+        const void *ptrs[] = {q, k, v, log_alpha, b, w, d_o, dq, dk, dv, d_log_alpha, db, dw};
+        for (const void *p : ptrs)
+            if (!p || !aligned16(p)) return GDR2_ERR_INVALID_ARG;
+    }
+    const void *opt[] = {init_state, d_final_state, d_init_state};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return GDR2_ERR_INVALID_ARG;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDR2_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDR2_OK;
+    const size_t need = gdr2::bwd_workspace_bytes(tokens, H, d_k, num_seqs);
+    if (!workspace || workspace_bytes < need) return GDR2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDR2_ERR_INVALID_ARG;
+    if (gdr2::bwd_slots(tokens, num_seqs) > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;
+
+    gdr2::BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w; a.d_o = d_o;
+    a.log_alpha = log_alpha;
+    a.init_state = init_state;
+    a.d_final = d_final_state;
+    a.cu_seqlens = cu_seqlens;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.db = db; a.dw = dw;
+    a.d_log_alpha = d_log_alpha;
+    a.d_init_state = d_init_state;
+    a.workspace = workspace;
+    a.B = B; a.T = T; a.H = H; a.d = d_k; a.num_seqs = num_seqs;
+    a.bf16 = dtype == GDR2_BF16;
+    return gdr2::launch_chunk_bwd(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
 gdr2_status gdr2_recurrent_step(const void *q, const void *k, const void *v,

@@ -66,6 +66,25 @@ cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
+// Gate-aware backward (bwd.cu): the vector-Jacobian product of the recurrence.
+struct BwdArgs {
+    const void *q, *k, *v, *b, *w, *d_o;
+    const float *log_alpha;
+    const float *init_state;    // may be null (zero)
+    const float *d_final;       // may be null (zero)
+    const int32_t *cu_seqlens;  // may be null
+    void *dq, *dk, *dv, *db, *dw;
+    float *d_log_alpha;
+    float *d_init_state;        // may be null
+    void *workspace;            // bwd_workspace_bytes(), 16-byte aligned
+    int64_t B, T, H, d, num_seqs;
+    bool bf16;
+};
+// Checkpoint slots (chunk-start states and chunk-end cotangents) of a batch.
+int64_t bwd_slots(int64_t tokens, int64_t num_seqs);
+size_t bwd_workspace_bytes(int64_t tokens, int64_t H, int64_t d, int64_t num_seqs);
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
+
 // Longest-first sequence order for packed batches (see order.cu).
 constexpr int kMaxSortSeqs = 16384;
 size_t order_bytes(int64_t num_seqs);

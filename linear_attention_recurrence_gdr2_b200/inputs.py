@@ -210,3 +210,18 @@ def preact_inputs(B: int, T: int, H: int, d: int, dtype: str = BF16, seed: int =
     if init_std is not None:
         s0 = (rng.standard_normal((B, H, d, d), dtype=np.float32) * np.float32(init_std)).astype(np.float32)
     return Inputs(q, k, v, la, b, w, s0, None, dtype, {"preact": True})
+
+
+def cotangents(inp: Inputs, seed: int = 1, final_std: float = 0.1):
+    """Seeded cotangents for the backward: d_o ~ N(0,1) shaped like o (rounded
+    to bf16 for bf16 workloads) and d_final ~ final_std * N(0,1), fp32
+    [N, H, dk, dv]. Draw order: d_o, d_final."""
+    rng = np.random.default_rng(seed)
+    B, T, H, dv = inp.v.shape
+    dk = inp.q.shape[-1]
+    d_o = rng.standard_normal((B, T, H, dv), dtype=np.float32)
+    if inp.dtype == BF16:
+        d_o = round_to_bf16(d_o)
+    d_final = (rng.standard_normal((inp.num_seqs, H, dk, dv), dtype=np.float32)
+               * np.float32(final_std)).astype(np.float32)
+    return d_o, d_final

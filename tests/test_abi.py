@@ -151,3 +151,47 @@ def test_prologue_flags_validated():
     assert L.gdr2_chunk_fwd_preact(*([None] * 8), 1, 64, 1, 64, 64, 1, 0, None, None, None, 0, 7,
                                    None) == INVALID
     assert gdr2.GDR2_PROLOGUE_ALL == 7
+
+
+def _bwd(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, s0=None, cu=None, do=FAKE, dsf=None,
+             B=2, T=128, H=4, dk=64, dv=64, N=2, dtype=0, dq=FAKE, dkk=FAKE, dvv=FAKE, dla=FAKE,
+             db=FAKE, dw=FAKE, ds0=None, ws=None, wsb=0, stream=None)
+    a.update(over)
+    return gdr2.lib().gdr2_chunk_bwd(
+        a["q"], a["k"], a["v"], a["la"], a["b"], a["w"], a["s0"], a["cu"], a["do"], a["dsf"],
+        a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dtype"], a["dq"], a["dkk"], a["dvv"],
+        a["dla"], a["db"], a["dw"], a["ds0"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_bwd_workspace_size():
+    """Two fp32 checkpoint arrays of (tokens/64 + N) slots and two per-token fp32 vectors."""
+    for B, T, H, d, N, cu in ((4, 2048, 16, 128, 4, False), (1, 1000, 3, 64, 5, True),
+                              (2, 1, 1, 64, 2, False), (1, 0, 2, 128, 3, True)):
+        need = gdr2.bwd_workspace_size(B, T, H, d, d, N, gdr2.GDR2_BF16)
+        slots = (B * T) // 64 + N
+        expect = 2 * slots * H * d * d * 4 + 2 * B * T * H * d * 4
+        assert need % 256 == 0 and expect <= need < expect + 256
+    with pytest.raises(gdr2.GDR2Error) as e:
+        gdr2.bwd_workspace_size(1, 64, 1, 96, 96, 1, gdr2.GDR2_FP32)
+    assert e.value.status == UNSUPPORTED
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(do=None), INVALID),
+    (dict(dla=None), INVALID),
+    (dict(dw=FAKE + 4), INVALID),
+    (dict(dsf=FAKE + 8), INVALID),
+    (dict(ds0=FAKE + 8), INVALID),
+    (dict(H=0), INVALID),
+    (dict(N=3), INVALID),
+    (dict(cu=FAKE, B=2), INVALID),
+    (dict(dtype=5), INVALID),
+    (dict(dk=128, dv=64), UNSUPPORTED),
+    ({}, WORKSPACE),                        # the workspace is required
+    (dict(ws=FAKE, wsb=1024), WORKSPACE),
+    (dict(ws=FAKE + 8, wsb=1 << 30), INVALID),
+    (dict(B=0, N=0, q=None, dq=None), OK),  # nothing to do
+])
+def test_chunk_bwd_rejects_bad_arguments(over, expect):
+    assert _bwd(**over) == expect

@@ -1,0 +1,116 @@
+"""The backward decomposition the CUDA kernels implement, checked in fp64
+against the oracle's reverse loop (CPU; no GPU, no import of the CUDA path).
+
+The vector-Jacobian product of the token recurrence ("Chunkwise training and
+gate-aware backward", ainews.random.gg article on Gated DeltaNet-2) is split
+into three sweeps:
+  A. forward, per value column: u_t = z_t - (alpha_t . S_{t-1})^T e_t and the
+     state at every chunk start (and after the last token);
+  B. reverse, per value column: the state cotangent G (from d_final), with
+     H_t = G + q_t do_t^T, du_t = H_t^T k_t, G <- alpha_t . (H_t - e_t du_t^T),
+     storing du_t and G at every chunk end; dv = du . w, dw = du . v, and the
+     last G is d_init_state;
+  C. per chunk and key row, given u, du and the two chunk checkpoints:
+     dq_t = S_t do_t, de_t = -(alpha_t . S_{t-1}) du_t, dkW_t = H_t u_t,
+     dk = dkW + b . de, db = k . de, and
+     dlog_alpha_t = sum_{s >= t in the chunk} (q.dq - k.dkW + e.de)_s
+                    + rowsum(G_end . S_end),
+     the last line because both recurrences telescope: the decay gradient of
+     token t equals that of token t+1 plus the three per-token terms, and at a
+     chunk end it is the row-wise product of the incoming cotangent with the
+     state there.
+Each sweep only needs reductions along one axis: A and B along key rows (per
+value column), C along value columns (per key row).
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+C = 64
+
+
+def sweeps(q, k, v, la, b, w, s0, do, dfin):
+    """One (sequence, head): q, k, la, b [T, dk]; v, w, do [T, dv]."""
+    T_len, dk = q.shape
+    dv_ = v.shape[1]
+    alpha, e, z = np.exp(la), b * k, w * v
+    nck = -(-T_len // C)
+    # sweep A
+    ck = np.zeros((nck + 1, dk, dv_))
+    U = np.zeros((T_len, dv_))
+    S = s0.copy()
+    for t in range(T_len):
+        if t % C == 0:
+            ck[t // C] = S
+        Sp = alpha[t][:, None] * S
+        U[t] = z[t] - Sp.T @ e[t]
+        S = Sp + np.outer(k[t], U[t])
+    ck[nck] = S
+    # sweep B
+    gk = np.zeros((nck, dk, dv_))
+    dU = np.zeros((T_len, dv_))
+    G = dfin.copy()
+    for t in range(T_len - 1, -1, -1):
+        if t == T_len - 1 or t % C == C - 1:
+            gk[t // C] = G
+        Hm = G + np.outer(q[t], do[t])
+        dU[t] = Hm.T @ k[t]
+        G = alpha[t][:, None] * (Hm - np.outer(e[t], dU[t]))
+    d_init = G
+    dvv, dww = dU * w, dU * v
+    # sweep C
+    dq, dkk, db, dla = (np.zeros((T_len, dk)) for _ in range(4))
+    for c in range(nck):
+        t0, t1 = c * C, min(T_len, (c + 1) * C)
+        dkW = np.zeros((t1 - t0, dk))
+        Hm = gk[c].copy()
+        for t in range(t1 - 1, t0 - 1, -1):          # pass R
+            Hm = Hm + np.outer(q[t], do[t])
+            dkW[t - t0] = Hm @ U[t]
+            Hm = alpha[t][:, None] * (Hm - np.outer(e[t], dU[t]))
+        S = ck[c].copy()
+        dg = np.zeros((t1 - t0, dk))
+        for t in range(t0, t1):                       # pass F
+            Sp = alpha[t][:, None] * S
+            de = -(Sp @ dU[t])
+            S = Sp + np.outer(k[t], U[t])
+            dq[t] = S @ do[t]
+            dkk[t] = dkW[t - t0] + b[t] * de
+            db[t] = k[t] * de
+            dg[t - t0] = q[t] * dq[t] - k[t] * dkW[t - t0] + e[t] * de
+        acc = np.sum(gk[c] * S, axis=1)               # rowsum(G_end . S_end)
+        for t in range(t1 - 1, t0 - 1, -1):
+            acc = acc + dg[t - t0]
+            dla[t] = acc
+    return dq, dkk, dvv, dla, db, dww, d_init
+
+
+def rel(a, b):
+    return np.abs(a - b).max() / max(1e-30, np.abs(b).max())
+
+
+@pytest.mark.parametrize("T,la_scale,with_state", [(200, 0.1, True), (64, 0.5, False), (1, 0.1, True),
+                                                   (130, 1.0, True)])
+def test_three_sweeps_match_oracle_backward(T, la_scale, with_state):
+    rng = np.random.default_rng(T)
+    dk, dv = 16, 12
+    q = rng.standard_normal((1, T, 1, dk))
+    k = rng.standard_normal((1, T, 1, dk))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, 1, dv))
+    la = -la_scale * np.log1p(np.exp(rng.standard_normal((1, T, 1, dk))))
+    b = 1 / (1 + np.exp(-rng.standard_normal((1, T, 1, dk))))
+    w = 1 / (1 + np.exp(-rng.standard_normal((1, T, 1, dv))))
+    s0 = 0.1 * rng.standard_normal((1, 1, dk, dv)) if with_state else None
+    do = rng.standard_normal((1, T, 1, dv))
+    dfin = rng.standard_normal((1, 1, dk, dv)) if with_state else np.zeros((1, 1, dk, dv))
+    ref = oracle.backward(q, k, v, la, b, w, s0, do, dfin)
+    s0_ = s0[0, 0] if with_state else np.zeros((dk, dv))
+    got = sweeps(q[0, :, 0], k[0, :, 0], v[0, :, 0], la[0, :, 0], b[0, :, 0], w[0, :, 0],
+                 s0_, do[0, :, 0], dfin[0, 0])
+    names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "d_init_state")
+    for name, g, r in zip(names, got, ref):
+        r = r[0, 0] if r.ndim == 4 and name == "d_init_state" else r[0, :, 0]
+        assert rel(g, r) < 1e-11, f"{name}: {rel(g, r):.2e}"

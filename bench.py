@@ -13,6 +13,9 @@ stream between barriers (max over ranks). In the same run:
                  heads (fp32 state 256 MiB), achieved HBM GB/s per step;
   * e2e       -- the same tokens/s with pinned host inputs copied in and o and
                  the final states copied out inside every timed step;
+  * backward  -- the gate-aware backward (gdr2_chunk_bwd) on the same batch:
+                 time per call and its fp32 CUDA-core flops against the SIMT
+                 fp32 peak (the kernels are ALU-bound);
   * cpu_baseline -- the fp64 oracle on the host cores (rank 0, N=1 only);
   * clocks    -- SM clock and throttle reasons sampled (NVML) while timing.
 Inputs are larger than L2 (268 MB of token tensors vs 126 MB), so the steps
@@ -92,6 +95,20 @@ def chunk_bytes(inp) -> int:
     per_token_head = el * (3 * dk + 2 * dv) + 4 * dk + el * dv
     state = inp.num_seqs * H * dk * dv * 4
     return ntok * H * per_token_head + state * (2 if inp.init_state is not None else 1)
+
+
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops (FMA) x 1.965 GHz
+SIMT_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops(inp) -> int:
+    """fp32 flops of one backward call per its three sweeps, per token-head and
+    state element: forward sweep 5 (decay, read, write), reverse sweep 7
+    (output term, du, decayed erase), per-chunk rows 14 (7 per pass)."""
+    ntok = inp.q.shape[0] * inp.q.shape[1]
+    H, dk = inp.q.shape[2], inp.q.shape[3]
+    dv = inp.v.shape[3]
+    return 26 * ntok * H * dk * dv
 
 
 def decode_bytes(N, H, dk, dv, el=2) -> int:
@@ -244,6 +261,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-calls", type=int, default=5)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -366,6 +385,37 @@ def main():
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "ms_per_step": e2e_ms}
 
+        # Backward on the same batch (after everything above: it reuses o's dtype for d_o).
+        bwd = None
+        if not args.no_backward:
+            gen_do, gen_df = gen.cotangents(inp, seed=7)
+            d_o = torch.from_numpy(gen_do).to(dev, tdt)
+            d_fin = torch.from_numpy(gen_df).to(dev)
+            bws = torch.empty(gdr2.bwd_workspace_size(B, T, H, d, d, N, dcode), dtype=torch.uint8,
+                              device=dev)
+
+            def bstep():
+                return gdr2.chunk_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["log_alpha"], dv_["b"],
+                                      dv_["w"], d_o, s0, d_fin, cu, workspace=bws)
+
+            for _ in range(3):
+                bstep()
+            barrier()
+            bev = [torch.cuda.Event(enable_timing=True) for _ in range(args.backward_calls + 1)]
+            bev[0].record(stream)
+            for i in range(args.backward_calls):
+                bstep()
+                bev[i + 1].record(stream)
+            barrier()
+            bper = [bev[i].elapsed_time(bev[i + 1]) for i in range(args.backward_calls)]
+            bms = statistics.mean(bper)
+            fl = bwd_flops(inp)
+            bwd = {"kernels": "column sweeps + per-chunk rows (2 launches)", "calls": args.backward_calls,
+                   "us_per_call": bms * 1e3, "tokens_per_s": inp.num_tokens / (bms * 1e-3),
+                   "bound": "alu", "flops_per_call": fl, "achieved_tflops": fl / (bms * 1e-3) / 1e12,
+                   "peak_tflops": SIMT_FP32_TFLOPS, "frac": fl / (bms * 1e-3) / 1e12 / SIMT_FP32_TFLOPS,
+                   "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz"}
+
     ms_per_step = total_ms / args.steps
     value = aggregate_throughput(inp.num_tokens, world, ms_per_step)
     kern_ms = statistics.mean(per)
@@ -404,6 +454,8 @@ def main():
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if bwd is not None:
+        line["backward"] = bwd
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp, label)
     print(json.dumps(line), flush=True)

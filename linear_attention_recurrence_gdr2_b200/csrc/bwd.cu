@@ -82,10 +82,34 @@ __device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16 *p, float a,
     *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
 }
 
+// ROWS consecutive floats from shared memory (16-byte aligned) as float4 loads.
+template <int ROWS>
+__device__ __forceinline__ void load_rows(const float *src, float (&out)[ROWS])
+{
+    static_assert(ROWS % 4 == 0, "rows come in float4 groups");
+#pragma unroll
+    for (int g = 0; g < ROWS / 4; ++g) {
+        const float4 v = *reinterpret_cast<const float4 *>(src + 4 * g);
+        out[4 * g] = v.x; out[4 * g + 1] = v.y; out[4 * g + 2] = v.z; out[4 * g + 3] = v.w;
+    }
+}
+
+// 16-byte asynchronous copy global -> shared (cp.async, bypassing L1).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
 // Sweeps A (blockIdx.z == 0) and B (blockIdx.z == 1). CTA = (sequence, head,
 // tile of 32 value columns); lane l of warp w owns columns 32*tile + 4w +
-// 2*(l/16) + {0,1} and key rows (l % 16) + 16m, so the reductions over key rows
-// are four xor-shuffles inside a half-warp. Row inputs (alpha, e, k, q) for 16
+// 2*(l/16) + {0,1} and the D/16 consecutive key rows starting at (l % 16) * D/16
+// (read from shared memory as float4), so the reductions over key rows are four
+// xor-shuffles inside a half-warp. Row inputs (alpha, e, k, q) for 16
 // tokens are staged in shared memory, the next 16 prefetched into registers
 // while the current ones are consumed.
 template <typename Tin, int D>
@@ -95,7 +119,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     constexpr int PF = kSub * D / kScanThreads;           // staged row elements per thread
     constexpr int PC = kSub * kTile / kScanThreads;       // staged column elements per thread
     static_assert(PF * kScanThreads == kSub * D && PC * kScanThreads == kSub * kTile, "staging split");
-    __shared__ float s_al[kSub * D], s_e[kSub * D], s_k[kSub * D], s_q[kSub * D];
+    __shared__ __align__(16) float s_al[kSub * D], s_e[kSub * D], s_k[kSub * D], s_q[kSub * D];
     __shared__ float s_c[3][kSub * kTile];   // A: z | B: do, v, w
 
     const int64_t n = blockIdx.x / p.H;
@@ -103,7 +127,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     const int tile = blockIdx.y;
     const bool rev = blockIdx.z != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rho = lane & 15;
+    const int row0 = (lane & 15) * ROWS;         // first of this lane's key rows
     const int jl = warp * 4 + (lane >> 4) * 2;   // first of this lane's two columns, in the tile
     const int j = tile * kTile + jl;
     const Tin *Q = static_cast<const Tin *>(p.q), *K = static_cast<const Tin *>(p.k);
@@ -116,13 +140,13 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     const int64_t nsub = (len + kSub - 1) / kSub;
     const int64_t head_state = (n * p.H + h) * (int64_t)D * D;
 
-    // X: state columns (A) or cotangent columns (B), rows rho + 16m
+    // X: state columns (A) or cotangent columns (B), rows row0 .. row0 + ROWS - 1
     float X0[ROWS], X1[ROWS];
     const float *x_init = rev ? p.d_final : p.init_state;
 #pragma unroll
     for (int m = 0; m < ROWS; ++m) {
         if (x_init) {
-            const float2 v2 = *reinterpret_cast<const float2 *>(x_init + head_state + (int64_t)(rho + 16 * m) * D + j);
+            const float2 v2 = *reinterpret_cast<const float2 *>(x_init + head_state + (int64_t)(row0 + m) * D + j);
             X0[m] = v2.x;
             X1[m] = v2.y;
         } else {
@@ -197,18 +221,19 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
             float *dst = (rev ? p.gk : p.ck) + ((base + chunk) * p.H + h) * (int64_t)D * D;
 #pragma unroll
             for (int m = 0; m < ROWS; ++m)
-                *reinterpret_cast<float2 *>(dst + (int64_t)(rho + 16 * m) * D + j) = make_float2(X0[m], X1[m]);
+                *reinterpret_cast<float2 *>(dst + (int64_t)(row0 + m) * D + j) = make_float2(X0[m], X1[m]);
         }
 
         if (!rev) {
             for (int tt = 0; tt < L; ++tt) {
                 const int64_t tok = start + sb * kSub + tt;
-                float r0 = 0.f, r1 = 0.f, kk[ROWS];
+                float r0 = 0.f, r1 = 0.f, al[ROWS], ee[ROWS], kk[ROWS];
+                load_rows<ROWS>(s_al + tt * D + row0, al);
+                load_rows<ROWS>(s_e + tt * D + row0, ee);
+                load_rows<ROWS>(s_k + tt * D + row0, kk);
 #pragma unroll
                 for (int m = 0; m < ROWS; ++m) {
-                    const int i = tt * D + rho + 16 * m;
-                    const float a = s_al[i], e = s_e[i];
-                    kk[m] = s_k[i];
+                    const float a = al[m], e = ee[m];
                     X0[m] *= a;                       // S' = Diag(alpha) S
                     X1[m] *= a;
                     r0 = fmaf(X0[m], e, r0);          // r = S'^T e
@@ -225,7 +250,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
                     X0[m] = fmaf(kk[m], u0, X0[m]);   // S = S' + k u^T
                     X1[m] = fmaf(kk[m], u1, X1[m]);
                 }
-                if (rho == 0)
+                if ((lane & 15) == 0)
                     *reinterpret_cast<float2 *>(p.U + (tok * p.H + h) * D + j) = make_float2(u0, u1);
             }
         } else {
@@ -233,11 +258,14 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
                 const int64_t tok = start + sb * kSub + tt;
                 const int c = tt * kTile + jl;
                 const float o0 = s_c[0][c], o1 = s_c[0][c + 1];
-                float d0 = 0.f, d1 = 0.f;
+                float d0 = 0.f, d1 = 0.f, qq[ROWS], kk[ROWS], al[ROWS], ee[ROWS];
+                load_rows<ROWS>(s_q + tt * D + row0, qq);
+                load_rows<ROWS>(s_k + tt * D + row0, kk);
+                load_rows<ROWS>(s_al + tt * D + row0, al);
+                load_rows<ROWS>(s_e + tt * D + row0, ee);
 #pragma unroll
                 for (int m = 0; m < ROWS; ++m) {
-                    const int i = tt * D + rho + 16 * m;
-                    const float qi = s_q[i], ki = s_k[i];
+                    const float qi = qq[m], ki = kk[m];
                     X0[m] = fmaf(qi, o0, X0[m]);      // H = G + q do^T
                     X1[m] = fmaf(qi, o1, X1[m]);
                     d0 = fmaf(X0[m], ki, d0);         // du = H^T k
@@ -250,12 +278,11 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
                 }
 #pragma unroll
                 for (int m = 0; m < ROWS; ++m) {
-                    const int i = tt * D + rho + 16 * m;
-                    const float a = s_al[i], e = s_e[i];
+                    const float a = al[m], e = ee[m];
                     X0[m] = a * fmaf(-e, d0, X0[m]);  // G = Diag(alpha)(H - e du^T)
                     X1[m] = a * fmaf(-e, d1, X1[m]);
                 }
-                if (rho == 0) {
+                if ((lane & 15) == 0) {
                     const int64_t off = (tok * p.H + h) * D + j;
                     *reinterpret_cast<float2 *>(p.dU + off) = make_float2(d0, d1);
                     store2(static_cast<Tin *>(p.dv) + off, d0 * s_c[2][c], d1 * s_c[2][c + 1]);  // du . w
@@ -267,20 +294,33 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     if (rev && p.d_init) {
 #pragma unroll
         for (int m = 0; m < ROWS; ++m)
-            *reinterpret_cast<float2 *>(p.d_init + head_state + (int64_t)(rho + 16 * m) * D + j) =
+            *reinterpret_cast<float2 *>(p.d_init + head_state + (int64_t)(row0 + m) * D + j) =
                 make_float2(X0[m], X1[m]);
     }
 }
 
 // Sweep C. CTA = (checkpoint slot, head); thread = (key rows rg + 64r, lane s
 // of 4), lane s holding value columns 4(s + 4g) .. +3. Row reductions over
-// value columns are two xor-shuffles inside each group of 4 lanes.
+// value columns are two xor-shuffles inside each group of 4 lanes. The chunk's
+// u, du and dO rows are copied to shared memory once (cp.async) and read from
+// there by both passes; the per-row scalars of the next token are loaded while
+// the current one is processed.
+template <typename Tin, int D>
+constexpr size_t rows_smem_bytes()
+{
+    return (size_t)kChunk * D * (3 * sizeof(float) + sizeof(Tin));
+}
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
 {
     constexpr int RPT = D / 64;   // key rows per thread
     constexpr int NG = D / 16;    // float4 column groups per thread
-    __shared__ float s_g[kChunk][D];   // dkW of the chunk, then the per-token decay terms
+    extern __shared__ __align__(16) unsigned char rows_smem[];
+    float *s_u = reinterpret_cast<float *>(rows_smem);   // [kChunk][D] u
+    float *s_du = s_u + kChunk * D;                       // [kChunk][D] du
+    float *s_g = s_du + kChunk * D;                       // [kChunk][D] dkW, then the decay terms
+    Tin *s_do = reinterpret_cast<Tin *>(s_g + kChunk * D);  // [kChunk][D] dO
 
     const int64_t slot = blockIdx.x;
     const int h = blockIdx.y;
@@ -305,6 +345,25 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
     const Tin *Bg = static_cast<const Tin *>(p.b), *DO = static_cast<const Tin *>(p.d_o);
     const int64_t slot_off = (slot * p.H + h) * (int64_t)D * D;
 
+    // stage u, du (fp32) and dO (Tin) of the chunk's L tokens
+    {
+        constexpr int F4 = D / 4;                       // 16-byte pieces per fp32 row
+        constexpr int T16 = D * (int)sizeof(Tin) / 16;  // 16-byte pieces per dO row
+        for (int idx = tid; idx < L * F4; idx += kRowThreads) {
+            const int tt = idx / F4, q4 = idx % F4;
+            const int64_t g = ((t0 + tt) * p.H + h) * D + 4 * q4;
+            cp_async16(s_u + tt * D + 4 * q4, p.U + g);
+            cp_async16(s_du + tt * D + 4 * q4, p.dU + g);
+        }
+        for (int idx = tid; idx < L * T16; idx += kRowThreads) {
+            const int tt = idx / T16, q16 = idx % T16;
+            constexpr int E = 16 / (int)sizeof(Tin);    // elements per piece
+            cp_async16(s_do + tt * D + E * q16, DO + ((t0 + tt) * p.H + h) * D + E * q16);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+    }
+
     float X[RPT][NG][4];
     // pass R: H from the chunk-end cotangent, tokens in reverse
 #pragma unroll
@@ -314,24 +373,37 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
             const float4 v4 = *reinterpret_cast<const float4 *>(p.gk + slot_off + (int64_t)(rg + 64 * r) * D + 4 * (s + 4 * g));
             X[r][g][0] = v4.x; X[r][g][1] = v4.y; X[r][g][2] = v4.z; X[r][g][3] = v4.w;
         }
-    for (int tt = L - 1; tt >= 0; --tt) {
+    // per-row scalars of the next token to process (prefetched one token ahead)
+    float nq[RPT], nk[RPT], nb[RPT], nla[RPT];
+    auto load_scalars = [&](int tt) {
         const int64_t row0 = ((t0 + tt) * p.H + h) * D;
-        float qr[RPT], ar[RPT], er[RPT], acc[RPT];
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
             const int64_t o = row0 + rg + 64 * r;
-            qr[r] = to_f32(Q[o]);
-            ar[r] = expf(p.la[o]);
-            er[r] = to_f32(Bg[o]) * to_f32(K[o]);
+            nq[r] = to_f32(Q[o]);
+            nk[r] = to_f32(K[o]);
+            nb[r] = to_f32(Bg[o]);
+            nla[r] = p.la[o];
+        }
+    };
+    load_scalars(L - 1);
+    for (int tt = L - 1; tt >= 0; --tt) {
+        float qr[RPT], ar[RPT], er[RPT], acc[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            qr[r] = nq[r];
+            ar[r] = expf(nla[r]);
+            er[r] = nb[r] * nk[r];
             acc[r] = 0.f;
         }
+        if (tt > 0) load_scalars(tt - 1);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             const int col = 4 * (s + 4 * g);
             float o4[4];
-            load_vec<Tin, 4>(DO + row0 + col, o4);
-            const float4 u4 = *reinterpret_cast<const float4 *>(p.U + row0 + col);
-            const float4 d4 = *reinterpret_cast<const float4 *>(p.dU + row0 + col);
+            load_vec<Tin, 4>(s_do + tt * D + col, o4);
+            const float4 u4 = *reinterpret_cast<const float4 *>(s_u + tt * D + col);
+            const float4 d4 = *reinterpret_cast<const float4 *>(s_du + tt * D + col);
             const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int r = 0; r < RPT; ++r)
@@ -346,7 +418,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
         for (int r = 0; r < RPT; ++r) {
             acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
             acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 2);
-            if (s == 0) s_g[tt][rg + 64 * r] = acc[r];
+            if (s == 0) s_g[tt * D + rg + 64 * r] = acc[r];
         }
     }
     __syncwarp();
@@ -360,26 +432,27 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
             X[r][g][0] = v4.x; X[r][g][1] = v4.y; X[r][g][2] = v4.z; X[r][g][3] = v4.w;
         }
     Tin *DQ = static_cast<Tin *>(p.dq), *DK = static_cast<Tin *>(p.dk), *DB = static_cast<Tin *>(p.db);
+    load_scalars(0);
     for (int tt = 0; tt < L; ++tt) {
         const int64_t row0 = ((t0 + tt) * p.H + h) * D;
         float qr[RPT], kr[RPT], br[RPT], ar[RPT], de[RPT], dq[RPT];
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
-            const int64_t o = row0 + rg + 64 * r;
-            qr[r] = to_f32(Q[o]);
-            kr[r] = to_f32(K[o]);
-            br[r] = to_f32(Bg[o]);
-            ar[r] = expf(p.la[o]);
+            qr[r] = nq[r];
+            kr[r] = nk[r];
+            br[r] = nb[r];
+            ar[r] = expf(nla[r]);
             de[r] = 0.f;
             dq[r] = 0.f;
         }
+        if (tt + 1 < L) load_scalars(tt + 1);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             const int col = 4 * (s + 4 * g);
             float o4[4];
-            load_vec<Tin, 4>(DO + row0 + col, o4);
-            const float4 u4 = *reinterpret_cast<const float4 *>(p.U + row0 + col);
-            const float4 d4 = *reinterpret_cast<const float4 *>(p.dU + row0 + col);
+            load_vec<Tin, 4>(s_do + tt * D + col, o4);
+            const float4 u4 = *reinterpret_cast<const float4 *>(s_u + tt * D + col);
+            const float4 d4 = *reinterpret_cast<const float4 *>(s_du + tt * D + col);
             const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int r = 0; r < RPT; ++r)
@@ -399,7 +472,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
             dq[r] += __shfl_xor_sync(0xffffffffu, dq[r], 1);
             dq[r] += __shfl_xor_sync(0xffffffffu, dq[r], 2);
             const float dev = -de[r];
-            const float dkw = s_g[tt][rg + 64 * r];
+            const float dkw = s_g[tt * D + rg + 64 * r];
             dkv[r] = fmaf(br[r], dev, dkw);                       // dk = dkW + b . de
             dbv[r] = kr[r] * dev;                                 // db = k . de
             dgv[r] = qr[r] * dq[r] - kr[r] * dkw + br[r] * kr[r] * dev;  // q.dq - k.dkW + e.de
@@ -411,7 +484,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
             if (s == 0) DQ[o] = from_f32<Tin>(dq[r]);
             else if (s == 1) DK[o] = from_f32<Tin>(dkv[r]);
             else if (s == 2) DB[o] = from_f32<Tin>(dbv[r]);
-            else s_g[tt][rg + 64 * r] = dgv[r];
+            else s_g[tt * D + rg + 64 * r] = dgv[r];
         }
     }
     // rowsum(G_end . S_end), then the reverse cumulative sum of the decay terms
@@ -436,7 +509,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) bwd_rows_kernel(BwdParams p)
         if (s == r) {
             float acc = bt[r];
             for (int tt = L - 1; tt >= 0; --tt) {
-                acc += s_g[tt][rg + 64 * r];
+                acc += s_g[tt * D + rg + 64 * r];
                 p.dla[((t0 + tt) * p.H + h) * D + rg + 64 * r] = acc;
             }
         }
@@ -453,8 +526,12 @@ cudaError_t launch_typed(const BwdParams &p, int64_t slots, cudaStream_t stream)
         if (e != cudaSuccess) return e;
     }
     if (p.tokens > 0) {
+        constexpr size_t smem = rows_smem_bytes<Tin, D>();
+        cudaError_t e = cudaFuncSetAttribute(bwd_rows_kernel<Tin, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
         dim3 grid((unsigned)slots, (unsigned)p.H);
-        bwd_rows_kernel<Tin, D><<<grid, kRowThreads, 0, stream>>>(p);
+        bwd_rows_kernel<Tin, D><<<grid, kRowThreads, smem, stream>>>(p);
         return cudaGetLastError();
     }
     return cudaSuccess;

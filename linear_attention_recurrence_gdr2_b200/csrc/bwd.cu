@@ -36,9 +36,9 @@
 namespace gdr2 {
 namespace {
 
-constexpr int kSub = 16;           // tokens staged per round of the column sweeps
-constexpr int kScanThreads = 256;  // 8 warps; a half-warp per pair of value columns
-constexpr int kTile = 32;          // value columns per column-sweep CTA
+constexpr int kSub = 8;            // tokens staged per round of the column sweeps
+constexpr int kScanThreads = 256;  // 8 warps; a half-warp per 4 value columns
+constexpr int kTile = 64;          // value columns per column-sweep CTA
 constexpr int kRowThreads = 256;   // 4 lanes per key row in the per-chunk kernel
 
 struct BwdParams {
@@ -106,29 +106,32 @@ __device__ __forceinline__ void cp_async_wait_all()
 }
 
 // Sweeps A (blockIdx.z == 0) and B (blockIdx.z == 1). CTA = (sequence, head,
-// tile of 32 value columns); lane l of warp w owns columns 32*tile + 4w +
-// 2*(l/16) + {0,1} and the D/16 consecutive key rows starting at (l % 16) * D/16
-// (read from shared memory as float4), so the reductions over key rows are four
-// xor-shuffles inside a half-warp. Row inputs (alpha, e, k, q) for 16
-// tokens are staged in shared memory, the next 16 prefetched into registers
-// while the current ones are consumed.
+// tile of 64 value columns); lane l of warp w owns the 4 columns 64*tile + 8w +
+// 4*(l/16) + {0..3} and the D/16 consecutive key rows starting at (l % 16) *
+// D/16 (read from shared memory as float4), so the reductions over key rows are
+// four xor-shuffles inside a half-warp, four independent columns at a time. One
+// CTA per 64 columns keeps both sweeps of a layer-sized batch resident at once.
+// Row inputs (alpha, e, k, q) for 8 tokens are staged in shared memory, the
+// next 8 prefetched into registers while the current ones are consumed.
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
 {
     constexpr int ROWS = D / 16;
+    constexpr int NC = 4;                                 // value columns per lane
     constexpr int PF = kSub * D / kScanThreads;           // staged row elements per thread
     constexpr int PC = kSub * kTile / kScanThreads;       // staged column elements per thread
     static_assert(PF * kScanThreads == kSub * D && PC * kScanThreads == kSub * kTile, "staging split");
+    static_assert(kTile == 8 * 2 * NC, "8 warps x 2 half-warps x NC columns");
     __shared__ __align__(16) float s_al[kSub * D], s_e[kSub * D], s_k[kSub * D], s_q[kSub * D];
-    __shared__ float s_c[3][kSub * kTile];   // A: z | B: do, v, w
+    __shared__ __align__(16) float s_c[3][kSub * kTile];   // A: z | B: do, v, w
 
     const int64_t n = blockIdx.x / p.H;
     const int h = (int)(blockIdx.x % p.H);
     const int tile = blockIdx.y;
     const bool rev = blockIdx.z != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row0 = (lane & 15) * ROWS;         // first of this lane's key rows
-    const int jl = warp * 4 + (lane >> 4) * 2;   // first of this lane's two columns, in the tile
+    const int row0 = (lane & 15) * ROWS;            // first of this lane's key rows
+    const int jl = warp * 2 * NC + (lane >> 4) * NC;  // first of this lane's columns, in the tile
     const int j = tile * kTile + jl;
     const Tin *Q = static_cast<const Tin *>(p.q), *K = static_cast<const Tin *>(p.k);
     const Tin *Bg = static_cast<const Tin *>(p.b), *V = static_cast<const Tin *>(p.v);
@@ -141,18 +144,13 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     const int64_t head_state = (n * p.H + h) * (int64_t)D * D;
 
     // X: state columns (A) or cotangent columns (B), rows row0 .. row0 + ROWS - 1
-    float X0[ROWS], X1[ROWS];
+    float X[NC][ROWS];
     const float *x_init = rev ? p.d_final : p.init_state;
 #pragma unroll
     for (int m = 0; m < ROWS; ++m) {
-        if (x_init) {
-            const float2 v2 = *reinterpret_cast<const float2 *>(x_init + head_state + (int64_t)(row0 + m) * D + j);
-            X0[m] = v2.x;
-            X1[m] = v2.y;
-        } else {
-            X0[m] = 0.f;
-            X1[m] = 0.f;
-        }
+        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (x_init) v4 = *reinterpret_cast<const float4 *>(x_init + head_state + (int64_t)(row0 + m) * D + j);
+        X[0][m] = v4.x; X[1][m] = v4.y; X[2][m] = v4.z; X[3][m] = v4.w;
     }
 
     float pf_la[PF], pf_k[PF], pf_b[PF], pf_q[PF], pc0[PC], pc1[PC], pc2[PC];
@@ -190,6 +188,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
         }
     };
 
+    constexpr int kSubPerChunk = kChunk / kSub;
     if (nsub > 0) prefetch(rev ? nsub - 1 : 0);
     for (int64_t it = 0; it < nsub; ++it) {
         const int64_t sb = rev ? nsub - 1 - it : it;
@@ -213,80 +212,81 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
         if (rev ? sb > 0 : sb + 1 < nsub) prefetch(rev ? sb - 1 : sb + 1);
 
         const int L = (int)((len - sb * kSub) < kSub ? (len - sb * kSub) : kSub);
-        const int64_t chunk = sb / (kChunk / kSub);
-        const bool at_chunk_edge = rev ? (sb % (kChunk / kSub) == kChunk / kSub - 1 || sb == nsub - 1)
-                                       : (sb % (kChunk / kSub) == 0);
+        const int64_t chunk = sb / kSubPerChunk;
+        const bool at_chunk_edge = rev ? (sb % kSubPerChunk == kSubPerChunk - 1 || sb == nsub - 1)
+                                       : (sb % kSubPerChunk == 0);
         if (at_chunk_edge) {
             // A: state at the chunk start; B: cotangent of the state at the chunk end
             float *dst = (rev ? p.gk : p.ck) + ((base + chunk) * p.H + h) * (int64_t)D * D;
 #pragma unroll
             for (int m = 0; m < ROWS; ++m)
-                *reinterpret_cast<float2 *>(dst + (int64_t)(row0 + m) * D + j) = make_float2(X0[m], X1[m]);
+                *reinterpret_cast<float4 *>(dst + (int64_t)(row0 + m) * D + j) =
+                    make_float4(X[0][m], X[1][m], X[2][m], X[3][m]);
         }
 
         if (!rev) {
             for (int tt = 0; tt < L; ++tt) {
                 const int64_t tok = start + sb * kSub + tt;
-                float r0 = 0.f, r1 = 0.f, al[ROWS], ee[ROWS], kk[ROWS];
+                float r[NC] = {0.f, 0.f, 0.f, 0.f}, al[ROWS], ee[ROWS], kk[ROWS];
                 load_rows<ROWS>(s_al + tt * D + row0, al);
                 load_rows<ROWS>(s_e + tt * D + row0, ee);
                 load_rows<ROWS>(s_k + tt * D + row0, kk);
 #pragma unroll
-                for (int m = 0; m < ROWS; ++m) {
-                    const float a = al[m], e = ee[m];
-                    X0[m] *= a;                       // S' = Diag(alpha) S
-                    X1[m] *= a;
-                    r0 = fmaf(X0[m], e, r0);          // r = S'^T e
-                    r1 = fmaf(X1[m], e, r1);
-                }
+                for (int m = 0; m < ROWS; ++m)
 #pragma unroll
-                for (int off = 8; off >= 1; off >>= 1) {
-                    r0 += __shfl_xor_sync(0xffffffffu, r0, off);
-                    r1 += __shfl_xor_sync(0xffffffffu, r1, off);
-                }
-                const float u0 = s_c[0][tt * kTile + jl] - r0, u1 = s_c[0][tt * kTile + jl + 1] - r1;
+                    for (int c = 0; c < NC; ++c) {
+                        X[c][m] *= al[m];                     // S' = Diag(alpha) S
+                        r[c] = fmaf(X[c][m], ee[m], r[c]);    // r = S'^T e
+                    }
 #pragma unroll
-                for (int m = 0; m < ROWS; ++m) {
-                    X0[m] = fmaf(kk[m], u0, X0[m]);   // S = S' + k u^T
-                    X1[m] = fmaf(kk[m], u1, X1[m]);
-                }
+                for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) r[c] += __shfl_xor_sync(0xffffffffu, r[c], off);
+                const float4 z4 = *reinterpret_cast<const float4 *>(&s_c[0][tt * kTile + jl]);
+                const float u[NC] = {z4.x - r[0], z4.y - r[1], z4.z - r[2], z4.w - r[3]};
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m)
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) X[c][m] = fmaf(kk[m], u[c], X[c][m]);   // S = S' + k u^T
                 if ((lane & 15) == 0)
-                    *reinterpret_cast<float2 *>(p.U + (tok * p.H + h) * D + j) = make_float2(u0, u1);
+                    *reinterpret_cast<float4 *>(p.U + (tok * p.H + h) * D + j) = make_float4(u[0], u[1], u[2], u[3]);
             }
         } else {
             for (int tt = L - 1; tt >= 0; --tt) {
                 const int64_t tok = start + sb * kSub + tt;
-                const int c = tt * kTile + jl;
-                const float o0 = s_c[0][c], o1 = s_c[0][c + 1];
-                float d0 = 0.f, d1 = 0.f, qq[ROWS], kk[ROWS], al[ROWS], ee[ROWS];
+                const int cb = tt * kTile + jl;
+                const float4 o4 = *reinterpret_cast<const float4 *>(&s_c[0][cb]);
+                const float oo[NC] = {o4.x, o4.y, o4.z, o4.w};
+                float d[NC] = {0.f, 0.f, 0.f, 0.f}, qq[ROWS], kk[ROWS], al[ROWS], ee[ROWS];
                 load_rows<ROWS>(s_q + tt * D + row0, qq);
                 load_rows<ROWS>(s_k + tt * D + row0, kk);
                 load_rows<ROWS>(s_al + tt * D + row0, al);
                 load_rows<ROWS>(s_e + tt * D + row0, ee);
 #pragma unroll
-                for (int m = 0; m < ROWS; ++m) {
-                    const float qi = qq[m], ki = kk[m];
-                    X0[m] = fmaf(qi, o0, X0[m]);      // H = G + q do^T
-                    X1[m] = fmaf(qi, o1, X1[m]);
-                    d0 = fmaf(X0[m], ki, d0);         // du = H^T k
-                    d1 = fmaf(X1[m], ki, d1);
-                }
+                for (int m = 0; m < ROWS; ++m)
 #pragma unroll
-                for (int off = 8; off >= 1; off >>= 1) {
-                    d0 += __shfl_xor_sync(0xffffffffu, d0, off);
-                    d1 += __shfl_xor_sync(0xffffffffu, d1, off);
-                }
+                    for (int c = 0; c < NC; ++c) {
+                        X[c][m] = fmaf(qq[m], oo[c], X[c][m]);   // H = G + q do^T
+                        d[c] = fmaf(X[c][m], kk[m], d[c]);       // du = H^T k
+                    }
 #pragma unroll
-                for (int m = 0; m < ROWS; ++m) {
-                    const float a = al[m], e = ee[m];
-                    X0[m] = a * fmaf(-e, d0, X0[m]);  // G = Diag(alpha)(H - e du^T)
-                    X1[m] = a * fmaf(-e, d1, X1[m]);
-                }
+                for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) d[c] += __shfl_xor_sync(0xffffffffu, d[c], off);
+#pragma unroll
+                for (int m = 0; m < ROWS; ++m)
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) X[c][m] = al[m] * fmaf(-ee[m], d[c], X[c][m]);  // G = Diag(alpha)(H - e du^T)
                 if ((lane & 15) == 0) {
                     const int64_t off = (tok * p.H + h) * D + j;
-                    *reinterpret_cast<float2 *>(p.dU + off) = make_float2(d0, d1);
-                    store2(static_cast<Tin *>(p.dv) + off, d0 * s_c[2][c], d1 * s_c[2][c + 1]);  // du . w
-                    store2(static_cast<Tin *>(p.dw) + off, d0 * s_c[1][c], d1 * s_c[1][c + 1]);  // du . v
+                    const float4 v4 = *reinterpret_cast<const float4 *>(&s_c[1][cb]);
+                    const float4 w4 = *reinterpret_cast<const float4 *>(&s_c[2][cb]);
+                    *reinterpret_cast<float4 *>(p.dU + off) = make_float4(d[0], d[1], d[2], d[3]);
+                    Tin *dvp = static_cast<Tin *>(p.dv) + off, *dwp = static_cast<Tin *>(p.dw) + off;
+                    store2(dvp, d[0] * w4.x, d[1] * w4.y);       // dv = du . w
+                    store2(dvp + 2, d[2] * w4.z, d[3] * w4.w);
+                    store2(dwp, d[0] * v4.x, d[1] * v4.y);       // dw = du . v
+                    store2(dwp + 2, d[2] * v4.z, d[3] * v4.w);
                 }
             }
         }
@@ -294,8 +294,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     if (rev && p.d_init) {
 #pragma unroll
         for (int m = 0; m < ROWS; ++m)
-            *reinterpret_cast<float2 *>(p.d_init + head_state + (int64_t)(row0 + m) * D + j) =
-                make_float2(X0[m], X1[m]);
+            *reinterpret_cast<float4 *>(p.d_init + head_state + (int64_t)(row0 + m) * D + j) =
+                make_float4(X[0][m], X[1][m], X[2][m], X[3][m]);
     }
 }
 

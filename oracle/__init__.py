@@ -4,15 +4,18 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package. The CUDA library never calls it and shares no
 code with it.
 
-The arithmetic lives in ``gdr2_oracle.c`` (plain sequential fp64 C, one token
-at a time); this module compiles it with gcc on first use and wraps it for
-numpy arrays. Every input is upcast to float64 before the call, so bf16 inputs
+The forward arithmetic lives in ``gdr2_oracle.c`` (plain sequential fp64 C,
+one token at a time); this module compiles it with gcc on first use and wraps
+it for numpy arrays. The backward (``backward``, the vector-Jacobian product
+of the same token rule) and the prologue are plain numpy in this module. Every input is upcast to float64 before the call, so bf16 inputs
 enter the oracle with exactly the values the GPU sees.
 
 Pinned by: tests/test_oracle_pins.py (KDA and Gated DeltaNet reductions,
 exact recall, b=0 closed form, brute-force transition products, the
 fast-weight argmin identity, state passing, varlen splitting, linearity; the
-prologue against scipy's logistic function, numpy's logaddexp and norm).
+prologue against scipy's logistic function, numpy's logaddexp and norm);
+tests/test_backward_oracle.py (the backward against central finite
+differences of the forward, linearity in the cotangents, planted mistakes).
 """
 from __future__ import annotations
 

@@ -21,6 +21,11 @@ into three sweeps:
      state there.
 Each sweep only needs reductions along one axis: A and B along key rows (per
 value column), C along value columns (per key row).
+
+The second half restates the same backward in the chunk (WY) form, with the
+forward's decay reference at chunk row 31: every per-chunk step is a product
+of 64-row tiles, and a chunk-to-chunk recurrence carries the state cotangent.
+It is checked against the oracle the same way.
 """
 import numpy as np
 import pytest
@@ -114,3 +119,99 @@ def test_three_sweeps_match_oracle_backward(T, la_scale, with_state):
     for name, g, r in zip(names, got, ref):
         r = r[0, 0] if r.ndim == 4 and name == "d_init_state" else r[0, :, 0]
         assert rel(g, r) < 1e-11, f"{name}: {rel(g, r):.2e}"
+
+
+# ---------------------------------------------------------------------------
+# The chunk (WY) form of the same backward: every per-chunk step is a dense
+# product of 64-row tiles, the form a tensor-core backward takes. With the
+# forward's chunk quantities (decay exponents d = g - g_31 about the chunk's
+# row 31, Qm = q e^d, Km = k e^-d, Em = e e^d, Sm = e^{g_31} S0, A, P, T and U)
+# and Ghat, the cotangent of the state at the chunk end:
+#   dU   = T^T (P^T dO + (Km . e^{d_end}) Ghat)            (du of every token)
+#   dQ   = e^d . (dO Sm^T + tril(dO U^T) Km)
+#   dE   = -e^d . (dU Sm^T + stril(dU U^T) Km)
+#   dKW  = e^-d . (triu(U dO^T) Qm - striu(U dU^T) Em) + e^{d_end - d} . (U Ghat^T)
+#   Ghat_prev = e^{g_31} . (Qm^T dO - Em^T dU) + e^{g_end} . Ghat
+# and the per-token combinations of the three-sweep form above (dk, db, the
+# decay terms, restarted at the chunk end with rowsum(Ghat . S_end)).
+MID = 31
+
+
+def inverse_unit_lower(A):
+    return np.linalg.solve(np.eye(A.shape[0]) + A, np.eye(A.shape[0]))
+
+
+def chunk_backward(q, k, v, la, b, w, s0, do, dfin):
+    T_len, dk = q.shape
+    dv_ = v.shape[1]
+    nck = -(-T_len // C)
+    pad = lambda x, t0, L: np.vstack([x[t0:t0 + L], np.zeros((C - L, x.shape[1]))])
+    # forward over chunks, keeping each chunk's quantities
+    S = s0.copy()
+    saved = []
+    for c in range(nck):
+        t0 = c * C
+        L = min(C, T_len - t0)
+        qc, kc, vc, lac, bc, wc, doc = (pad(x, t0, L) for x in (q, k, v, la, b, w, do))
+        g = np.cumsum(lac, axis=0)
+        d = g - g[MID]
+        qm, km, em = qc * np.exp(d), kc * np.exp(-d), bc * kc * np.exp(d)
+        sm = np.exp(g[MID])[:, None] * S
+        A = np.tril(em @ km.T, -1)
+        P = np.tril(qm @ km.T)
+        Tinv = inverse_unit_lower(A)
+        U = Tinv @ (wc * vc - em @ sm)
+        X = sm + km.T @ U                       # S_end = e^{d_end} . X
+        saved.append((t0, L, qc, kc, vc, bc, wc, doc, g, d, qm, km, em, sm, P, Tinv, U, X))
+        S = np.exp(d[C - 1])[:, None] * X
+    dq, dkk, db, dla = (np.zeros((T_len, dk)) for _ in range(4))
+    dvv, dww = np.zeros((T_len, dv_)), np.zeros((T_len, dv_))
+    Gh = dfin.copy()
+    for c in range(nck - 1, -1, -1):
+        t0, L, qc, kc, vc, bc, wc, doc, g, d, qm, km, em, sm, P, Tinv, U, X = saved[c]
+        ed = np.exp(d)
+        dend = d[C - 1]
+        dU = Tinv.T @ (P.T @ doc + (km * np.exp(dend)) @ Gh)
+        dQ = ed * (doc @ sm.T + np.tril(doc @ U.T) @ km)
+        dE = -ed * (dU @ sm.T + np.tril(dU @ U.T, -1) @ km)
+        dKW = (np.exp(-d) * (np.triu(U @ doc.T) @ qm - np.triu(U @ dU.T, 1) @ em)
+               + np.exp(dend - d) * (U @ Gh.T))
+        e = bc * kc
+        dg = qc * dQ - kc * dKW + e * dE
+        acc = np.exp(dend) * np.sum(Gh * X, axis=1)      # rowsum(Ghat . S_end)
+        for t in range(L - 1, -1, -1):
+            acc = acc + dg[t]
+            dla[t0 + t] = acc
+        dq[t0:t0 + L] = dQ[:L]
+        dkk[t0:t0 + L] = (dKW + bc * dE)[:L]
+        db[t0:t0 + L] = (kc * dE)[:L]
+        dvv[t0:t0 + L] = (dU * wc)[:L]
+        dww[t0:t0 + L] = (dU * vc)[:L]
+        Gh = np.exp(g[MID])[:, None] * (qm.T @ doc - em.T @ dU) + np.exp(g[C - 1])[:, None] * Gh
+    return dq, dkk, dvv, dla, db, dww, Gh
+
+
+@pytest.mark.parametrize("T,la_scale,with_state", [(200, 0.1, True), (64, 0.5, False), (1, 0.1, True),
+                                                   (130, 1.0, True), (31, 0.3, True)])
+def test_chunk_form_backward_matches_oracle(T, la_scale, with_state):
+    rng = np.random.default_rng(100 + T)
+    dk, dv = 16, 12
+    q = rng.standard_normal((1, T, 1, dk))
+    k = rng.standard_normal((1, T, 1, dk))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, 1, dv))
+    la = -la_scale * np.log1p(np.exp(rng.standard_normal((1, T, 1, dk))))
+    b = 1 / (1 + np.exp(-rng.standard_normal((1, T, 1, dk))))
+    w = 1 / (1 + np.exp(-rng.standard_normal((1, T, 1, dv))))
+    s0 = 0.1 * rng.standard_normal((1, 1, dk, dv)) if with_state else None
+    do = rng.standard_normal((1, T, 1, dv))
+    dfin = rng.standard_normal((1, 1, dk, dv)) if with_state else np.zeros((1, 1, dk, dv))
+    ref = oracle.backward(q, k, v, la, b, w, s0, do, dfin)
+    s0_ = s0[0, 0] if with_state else np.zeros((dk, dv))
+    got = chunk_backward(q[0, :, 0], k[0, :, 0], v[0, :, 0], la[0, :, 0], b[0, :, 0], w[0, :, 0],
+                         s0_, do[0, :, 0], dfin[0, 0])
+    names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "d_init_state")
+    for name, g, r in zip(names, got, ref):
+        r = r[0, 0] if name == "d_init_state" else r[0, :, 0]
+        assert rel(g, r) < 1e-10, f"{name}: {rel(g, r):.2e}"

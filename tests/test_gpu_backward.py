@@ -124,3 +124,13 @@ def test_bwd_layer_prefill_units(cuda_device):
         for name, g, r in zip(NAMES[:6], got[:6], ref[:6]):
             assert_close(f"layer unit({n},{h}) {name}", g[rows], r[0, :, 0], "bf16")
         assert_close(f"layer unit({n},{h}) d_init_state", got[6][n, h], ref[6][0, 0], "bf16")
+
+
+def test_bwd_deterministic(cuda_device):
+    """No atomics and a fixed reduction order: two calls agree bit for bit."""
+    inp = gen.make_inputs(2, 300, 4, 128, 128, "bf16", seed=21, init_std=0.05)
+    d_o, d_final = gen.cotangents(inp, seed=22)
+    a = run_bwd(inp, d_o, d_final, cuda_device)
+    b = run_bwd(inp, d_o, d_final, cuda_device)
+    for name, x, y in zip(NAMES, a, b):
+        assert np.array_equal(x, y), f"{name} differs between two identical calls"

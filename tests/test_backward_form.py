@@ -215,3 +215,99 @@ def test_chunk_form_backward_matches_oracle(T, la_scale, with_state):
     for name, g, r in zip(names, got, ref):
         r = r[0, 0] if name == "d_init_state" else r[0, :, 0]
         assert rel(g, r) < 1e-10, f"{name}: {rel(g, r):.2e}"
+
+
+# ---------------------------------------------------------------------------
+# Segment split of the two sweeps (for few long sequences). Both sweeps are
+# affine in their state, so a sequence cut into P segments can run every
+# segment at once and chain the segments afterwards:
+#   A: S_end(p) = Phi_p S_start(p) + S0_p, with Phi_p the product of the
+#      segment's transition matrices M_t = (I - k_t e_t^T) Diag(alpha_t);
+#      the segment run from the identity (z = 0) gives Phi_p and, per token,
+#      psi_t = Phi_{<t}^T (alpha_t . e_t), so that u_t = u0_t - S_start^T psi_t.
+#   B: G_start(p) = Phi_p^T G_end(p) + G0_p; the reverse run from the identity
+#      with dO = 0 gives Phi_p^T as its last cotangent and, as its du,
+#      chi_t = M_end ... M_{t+1} k_t, so that du_t = du0_t + G_end^T chi_t.
+# The chunk checkpoints follow the same way: a chunk-start state is the zero
+# run's plus the identity run's checkpoint times S_start, a chunk-end
+# cotangent the zero run's plus the identity run's times G_end.
+
+
+def sweep_a(alpha, e, k, z, s_init):
+    """Sweep A over a token range: per-token u and the state before each token."""
+    S = s_init.copy()
+    us, before = [], []
+    for t in range(alpha.shape[0]):
+        before.append(S)
+        Sp = alpha[t][:, None] * S
+        u = z[t] - Sp.T @ e[t]
+        S = Sp + np.outer(k[t], u)
+        us.append(u)
+    return np.array(us), np.array(before), S
+
+
+def sweep_b(alpha, e, k, q, do, g_init):
+    """Sweep B over a token range: per-token du and the cotangent after each token."""
+    G = g_init.copy()
+    dus, after = [None] * alpha.shape[0], [None] * alpha.shape[0]
+    for t in range(alpha.shape[0] - 1, -1, -1):
+        after[t] = G
+        Hm = G + np.outer(q[t], do[t])
+        dus[t] = Hm.T @ k[t]
+        G = alpha[t][:, None] * (Hm - np.outer(e[t], dus[t]))
+    return np.array(dus), np.array(after), G
+
+
+@pytest.mark.parametrize("T,P,la_scale", [(256, 4, 0.1), (200, 3, 0.5), (97, 2, 1.0)])
+def test_segment_split_of_the_sweeps(T, P, la_scale):
+    rng = np.random.default_rng(T + P)
+    dk, dv = 12, 10
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    alpha = np.exp(-la_scale * np.log1p(np.exp(rng.standard_normal((T, dk)))))
+    b = 1 / (1 + np.exp(-rng.standard_normal((T, dk))))
+    e = b * k
+    z = rng.standard_normal((T, dv))
+    do = rng.standard_normal((T, dv))
+    s0 = 0.1 * rng.standard_normal((dk, dv))
+    dfin = rng.standard_normal((dk, dv))
+    u_ref, st_ref, _ = sweep_a(alpha, e, k, z, s0)
+    du_ref, gt_ref, ginit_ref = sweep_b(alpha, e, k, q, do, dfin)
+
+    cuts = np.linspace(0, T, P + 1).astype(int)
+    I, zeros_z, zeros_do = np.eye(dk), np.zeros((T, dk)), np.zeros((T, dk))   # identity runs are dk wide
+    # every segment at once: from zero (A, B) and from the identity (z = 0, dO = 0)
+    segA, segB = [], []
+    for p in range(P):
+        a, c = cuts[p], cuts[p + 1]
+        sl = slice(a, c)
+        u0, b0, e0 = sweep_a(alpha[sl], e[sl], k[sl], z[sl], np.zeros((dk, dv)))
+        uI, bI, Phi = sweep_a(alpha[sl], e[sl], k[sl], zeros_z[sl], I)
+        segA.append((u0, b0, e0, -uI, bI, Phi))     # -uI[t] = psi_t (u from the identity, z = 0)
+        d0, a0, g0 = sweep_b(alpha[sl], e[sl], k[sl], q[sl], do[sl], np.zeros((dk, dv)))
+        chi, aI, PhiT = sweep_b(alpha[sl], e[sl], k[sl], q[sl], zeros_do[sl], I)
+        segB.append((d0, a0, g0, chi, aI, PhiT))
+    # chain the segments: A forward, B in reverse
+    s_start, g_end = [s0], [None] * P
+    for p in range(P - 1):
+        _, _, e0, _, _, Phi = segA[p]
+        s_start.append(Phi @ s_start[p] + e0)
+    g_end[P - 1] = dfin
+    for p in range(P - 1, 0, -1):
+        _, _, g0, _, _, PhiT = segB[p]
+        g_end[p - 1] = PhiT @ g_end[p] + g0
+    np.testing.assert_allclose(segB[0][5] @ g_end[0] + segB[0][2], ginit_ref, rtol=1e-11, atol=1e-11)
+    # per-token corrections and checkpoints
+    for p in range(P):
+        a, c = cuts[p], cuts[p + 1]
+        u0, b0, _, psi, bI, _ = segA[p]
+        d0, a0, _, chi, aI, _ = segB[p]
+        u = u0 - psi @ s_start[p]                    # u_t = u0_t - S_start^T psi_t
+        du = d0 + chi @ g_end[p]                     # du_t = du0_t + G_end^T chi_t
+        np.testing.assert_allclose(u, u_ref[a:c], rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(du, du_ref[a:c], rtol=1e-10, atol=1e-11)
+        before = b0 + np.einsum("tij,jv->tiv", bI, s_start[p])
+        after = a0 + np.einsum("tij,jv->tiv", aI, g_end[p])     # G_t = G0_t + G^I_t G_end
+        np.testing.assert_allclose(before, st_ref[a:c], rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(after, gt_ref[a:c], rtol=1e-10, atol=1e-11)

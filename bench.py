@@ -408,7 +408,7 @@ def main():
                 bev[i + 1].record(stream)
             barrier()
             bper = [bev[i].elapsed_time(bev[i + 1]) for i in range(args.backward_calls)]
-            bms = statistics.mean(bper)
+            bms = max_over_ranks(statistics.mean(bper))
             fl = bwd_flops(inp)
             bwd = {"kernels": "column sweeps + per-chunk rows (2 launches)", "calls": args.backward_calls,
                    "us_per_call": bms * 1e3, "tokens_per_s": inp.num_tokens / (bms * 1e-3),

@@ -251,6 +251,26 @@ def cpu_baseline(inp, label, wall_s=2.0):
                       f"{label} workload ({dt:.2f} s wall of fp64 work on {cores} threads)"}
 
 
+def cpu_backward_baseline(inp, d_o, label, tokens=512, heads=1):
+    """Times the fp64 backward oracle (oracle.backward, plain numpy) on the
+    host on a bounded sample: sequence 0, its first `tokens` tokens and
+    `heads` heads, with the benchmark's output cotangents and no final-state
+    cotangent. Reported in tokens/s of all H heads, like the GPU number."""
+    import oracle
+    B, T, H, d = inp.q.shape
+    tokens = min(tokens, T)
+    sl = lambda x: np.ascontiguousarray(x[:1, :tokens, :heads], dtype=np.float64)
+    arrs = [sl(x) for x in (inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w)]
+    s0 = (np.ascontiguousarray(inp.init_state[:1, :heads], dtype=np.float64)
+          if inp.init_state is not None else None)
+    t0 = time.perf_counter()
+    oracle.backward(*arrs, s0, sl(d_o), None)
+    dt = time.perf_counter() - t0
+    return {"value": tokens * heads / H / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"sequence 0, first {tokens} tokens, {heads} of {H} heads of the {label} "
+                      f"workload ({dt:.2f} s wall of fp64 numpy on one thread)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -458,6 +478,8 @@ def main():
         line["backward"] = bwd
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp, label)
+        if bwd is not None:
+            bwd["cpu_baseline"] = cpu_backward_baseline(inp, gen_do, label)
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -58,3 +58,16 @@ def test_single_process_reduce_is_identity():
     import bench
     assert bench.reduce_max(1.25) == 1.25
     assert bench.aggregate_throughput(100, 1, 2.0) == pytest.approx(50000.0)
+
+
+def test_cpu_backward_baseline_runs_on_a_small_sample():
+    """The backward's CPU baseline (the fp64 oracle on a bounded sample) runs
+    on the host and reports tokens/s of all heads."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from linear_attention_recurrence_gdr2_b200 import inputs as gen
+    inp = gen.make_inputs(2, 40, 4, 16, 16, "bf16", seed=3, init_std=0.1)
+    d_o, _ = gen.cotangents(inp)
+    r = bench.cpu_backward_baseline(inp, d_o, "tiny", tokens=32, heads=2)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+    assert "first 32 tokens, 2 of 4 heads" in r["sample"]

@@ -259,6 +259,8 @@ def cpu_backward_baseline(inp, d_o, label, tokens=512, heads=1):
     import oracle
     B, T, H, d = inp.q.shape
     tokens = min(tokens, T)
+    if inp.cu_seqlens is not None:   # stay inside the packed batch's first sequence
+        tokens = min(tokens, int(inp.cu_seqlens[1] - inp.cu_seqlens[0]))
     sl = lambda x: np.ascontiguousarray(x[:1, :tokens, :heads], dtype=np.float64)
     arrs = [sl(x) for x in (inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w)]
     s0 = (np.ascontiguousarray(inp.init_state[:1, :heads], dtype=np.float64)

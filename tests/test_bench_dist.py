@@ -71,3 +71,13 @@ def test_cpu_backward_baseline_runs_on_a_small_sample():
     r = bench.cpu_backward_baseline(inp, d_o, "tiny", tokens=32, heads=2)
     assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
     assert "first 32 tokens, 2 of 4 heads" in r["sample"]
+
+
+def test_cpu_backward_baseline_stays_in_the_first_packed_sequence():
+    sys.path.insert(0, ROOT)
+    import bench
+    from linear_attention_recurrence_gdr2_b200 import inputs as gen
+    inp = gen.make_inputs(1, 0, 2, 16, 16, "fp32", seed=4, init_std=0.1, lengths=[20, 50])
+    d_o, _ = gen.cotangents(inp)
+    r = bench.cpu_backward_baseline(inp, d_o, "tiny packed", tokens=512, heads=1)
+    assert "first 20 tokens" in r["sample"]

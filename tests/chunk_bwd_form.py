@@ -9,7 +9,8 @@ kernel that feeds bf16 or tf32 operands and accumulates in fp32:
 
 prints the relative L2 error of every gradient against the fp64 oracle for
 fp32, tf32 (10 mantissa bits, truncated) and bf16 (round to nearest even)
-operands, on one head of the layer shape (d = 128, bf16 inputs).
+operands, and for the two mixed choices (chains in one format, per-chunk row
+products in the other), on one head of the layer shape (d = 128, bf16 inputs).
 Formulas (decay exponents d = g - g_31 about chunk row 31, Qm = q e^d,
 Km = k e^-d, Em = b k e^d, Sm = e^{g_31} S0, Ghat the cotangent of the state at
 the chunk end):
@@ -44,10 +45,17 @@ def fp32(x):
     return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
-def chunk_backward(q, k, v, la, b, w, s0, do, dfin, rnd=None):
+def _product(rnd):
+    return (lambda a, c: a @ c) if rnd is None else (lambda a, c: fp32(rnd(a) @ rnd(c)))
+
+
+def chunk_backward(q, k, v, la, b, w, s0, do, dfin, rnd=None, rnd_rows="same"):
     """One (sequence, head): q, k, la, b [T, dk]; v, w, do [T, dv]; s0, dfin [dk, dv].
-    Returns dq, dk, dv, dlog_alpha, db, dw, d_init_state."""
-    mm = (lambda a, c: a @ c) if rnd is None else (lambda a, c: fp32(rnd(a) @ rnd(c)))
+    `rnd` rounds the operands of the chain products (A, P, U, dU, the state and
+    cotangent updates); `rnd_rows` those of the per-chunk row products (dQ, dE,
+    dKW), by default the same. Returns dq, dk, dv, dlog_alpha, db, dw, d_init_state."""
+    mm = _product(rnd)
+    mr = mm if rnd_rows == "same" else _product(rnd_rows)
     T_len, dk = q.shape
     dv_ = v.shape[1]
     nck = -(-T_len // C)
@@ -77,10 +85,10 @@ def chunk_backward(q, k, v, la, b, w, s0, do, dfin, rnd=None):
         ed = np.exp(d)
         dend = d[C - 1]
         dU = mm(Tinv.T, mm(P.T, doc) + mm(km * np.exp(dend), Gh))
-        dQ = ed * (mm(doc, sm.T) + mm(np.tril(mm(doc, U.T)), km))
-        dE = -ed * (mm(dU, sm.T) + mm(np.tril(mm(dU, U.T), -1), km))
-        dKW = (np.exp(-d) * (mm(np.triu(mm(U, doc.T)), qm) - mm(np.triu(mm(U, dU.T), 1), em))
-               + np.exp(dend - d) * mm(U, Gh.T))
+        dQ = ed * (mr(doc, sm.T) + mr(np.tril(mr(doc, U.T)), km))
+        dE = -ed * (mr(dU, sm.T) + mr(np.tril(mr(dU, U.T), -1), km))
+        dKW = (np.exp(-d) * (mr(np.triu(mr(U, doc.T)), qm) - mr(np.triu(mr(U, dU.T), 1), em))
+               + np.exp(dend - d) * mr(U, Gh.T))
         dg = qc * dQ - kc * dKW + bc * kc * dE
         acc = np.exp(dend) * np.sum(Gh * X, axis=1)         # rowsum(Ghat . S_end)
         for t in range(L - 1, -1, -1):
@@ -95,7 +103,7 @@ def chunk_backward(q, k, v, la, b, w, s0, do, dfin, rnd=None):
     return dq, dkk, dvv, dla, db, dww, Gh
 
 
-def operand_precision_errors(T=512, seed=3, rnd=tf32):
+def operand_precision_errors(T=512, seed=3, rnd=tf32, rnd_rows="same"):
     """Relative L2 error of every gradient of the rounded chunk form against
     the fp64 oracle, on one head of the layer shape with bf16 inputs."""
     import oracle
@@ -106,7 +114,7 @@ def operand_precision_errors(T=512, seed=3, rnd=tf32):
     f = lambda x: x[0, :, 0].astype(np.float64)
     got = chunk_backward(f(inp.q), f(inp.k), f(inp.v), f(inp.log_alpha), f(inp.b), f(inp.w),
                          inp.init_state[0, 0].astype(np.float64), f(d_o),
-                         d_f[0, 0].astype(np.float64), rnd)
+                         d_f[0, 0].astype(np.float64), rnd, rnd_rows)
     names = ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "d_init_state")
     out = {}
     for name, g, r in zip(names, got, ref):
@@ -119,6 +127,8 @@ if __name__ == "__main__":
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     sys.path.insert(0, root)
     T = int(sys.argv[1]) if len(sys.argv) > 1 else 512
-    for name, rnd in (("fp32", fp32), ("tf32", tf32), ("bf16", bf16)):
-        e = operand_precision_errors(T, rnd=rnd)
+    for name, rnd, rows in (("fp32", fp32, "same"), ("tf32", tf32, "same"), ("bf16", bf16, "same"),
+                            ("chains tf32, rows bf16", tf32, bf16),
+                            ("chains bf16, rows tf32", bf16, tf32)):
+        e = operand_precision_errors(T, rnd=rnd, rnd_rows=rows)
         print(name, " ".join(f"{k}={v:.1e}" for k, v in e.items()))

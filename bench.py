@@ -2,15 +2,26 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill|long|varlen] [--no-cpu-baseline]
+                    [--no-e2e] [--no-backward] [--no-extra-workloads]
 
 One step = one chunkwise forward (gdr2_chunk_fwd, bf16, H=16, d_k=d_v=128)
 over the layer-shaped prefill batch B=4 x T=2048 (8,192 tokens). The line's
-`value` is tokens/s over all ranks, timed with CUDA events on the launching
-stream between barriers (max over ranks). In the same run:
-  * roofline  -- algorithmic HBM bytes of one chunk-forward launch / its mean
-                 CUDA-event duration, against the measured copy bandwidth;
+`value` is tokens/s over all ranks: K steps back to back, timed with CUDA
+events on the launching stream between barriers (max over ranks), i.e. the
+mean step time. Every per-launch figure also carries its median, p10 and p90.
+In the same run:
+  * roofline  -- the chunk forward's bound: the slower of its algorithmic HBM
+                 bytes at the measured copy bandwidth and its algorithmic
+                 FLOPs at the measured bf16 tensor-core rate (the bytes, for
+                 this workload); achieved = bytes / median launch time;
+  * l2_flushed -- the same launch timed alone after overwriting a 256 MiB
+                 buffer (twice L2) before every launch;
+  * long, varlen -- a few launches of the long-context (T=32768, H=16) and
+                 packed variable-length (64 sequences) workloads, each with
+                 its own roofline;
   * decode    -- 64 consecutive gdr2_recurrent_step calls on N=256 x H=16
-                 heads (fp32 state 256 MiB), achieved HBM GB/s per step;
+                 heads (fp32 state 256 MiB), fresh token inputs every step,
+                 achieved HBM GB/s per step;
   * e2e       -- the same tokens/s with pinned host inputs copied in and o and
                  the final states copied out inside every timed step;
   * backward  -- the gate-aware backward (gdr2_chunk_bwd) on the same batch:
@@ -18,8 +29,8 @@ stream between barriers (max over ranks). In the same run:
                  fp32 peak (the kernels are ALU-bound);
   * cpu_baseline -- the fp64 oracle on the host cores (rank 0, N=1 only);
   * clocks    -- SM clock and throttle reasons sampled (NVML) while timing.
-Inputs are larger than L2 (268 MB of token tensors vs 126 MB), so the steps
-run back to back without an explicit flush.
+The prefill inputs (268 MB of token tensors) are larger than L2 (126 MB), so
+the back-to-back steps of the headline number run without a flush.
 
 Under torchrun every rank runs its own replica of the workload on its own GPU
 (the (sequence, head) units are independent: no collective on the data path;
@@ -116,6 +127,51 @@ def decode_bytes(N, H, dk, dv, el=2) -> int:
     return N * H * (2 * dk * dv * 4 + el * (3 * dk + 2 * dv) + 4 * dk + el * dv)
 
 
+def chunk_flops_per_chunk(d: int, C: int = 64) -> int:
+    """Algorithmic FLOPs of the chunk form for one (chunk, head), triangular
+    structure exploited: A = strict_tril(Ebar Kbar^T), P = tril(Qbar Kbar^T),
+    (I + A)^{-1} (C^3 / 3), W = T Ebar and U0 = T Z (unit lower-triangular T),
+    W S, Qbar S and (K e^{g_C - g})^T U (dense d x d), tril(P) U."""
+    strict, incl = C * (C - 1) // 2, C * (C + 1) // 2
+    return (strict * 2 * d + incl * 2 * d + C ** 3 // 3 + 2 * strict * 2 * d
+            + 3 * C * d * d * 2 + incl * 2 * d)
+
+
+def chunk_flops(inp) -> int:
+    """Algorithmic FLOPs of one chunk-forward launch: every chunk of every
+    sequence (a ragged last chunk counted whole, as the kernels run it)."""
+    H, d = inp.q.shape[2], inp.q.shape[3]
+    if inp.cu_seqlens is not None:
+        lengths = np.diff(np.asarray(inp.cu_seqlens, dtype=np.int64))
+        chunks = int(np.sum((lengths + 63) // 64))
+    else:
+        chunks = inp.q.shape[0] * ((inp.q.shape[1] + 63) // 64)
+    return chunks * H * chunk_flops_per_chunk(d)
+
+
+def stats_ms(per_ms):
+    """Mean, median, p10 and p90 of per-launch times (ms -> us)."""
+    xs = np.asarray(per_ms, dtype=np.float64) * 1e3
+    return {"mean_us": float(xs.mean()), "median_us": float(np.median(xs)),
+            "p10_us": float(np.percentile(xs, 10)), "p90_us": float(np.percentile(xs, 90))}
+
+
+def chunk_roofline(inp, us, hbm_peak, tflops_peak, peak_src):
+    """The chunk forward's roofline at a launch time of `us` microseconds: the
+    bound is the slower of bytes / HBM bandwidth and FLOPs / tensor rate."""
+    nbytes, flops = chunk_bytes(inp), chunk_flops(inp)
+    t_hbm = nbytes / (hbm_peak * 1e9) * 1e6
+    t_tc = flops / (tflops_peak * 1e12) * 1e6
+    hbm = t_hbm >= t_tc
+    achieved = nbytes / (us * 1e-6) / 1e9 if hbm else flops / (us * 1e-6) / 1e12
+    peak = hbm_peak if hbm else tflops_peak
+    return {"bound": "hbm" if hbm else "tensor", "achieved": achieved, "peak": peak,
+            "unit": "GB/s" if hbm else "TFLOP/s", "frac": achieved / peak,
+            "bytes_per_launch": nbytes, "flops_per_launch": flops,
+            "t_hbm_us": t_hbm, "t_tensor_us": t_tc,
+            "tensor_peak_tflops": tflops_peak, "peak_source": peak_src}
+
+
 class ClockSampler:
     """Samples the SM clock and throttle reasons through NVML in a thread."""
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -164,6 +220,15 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b],
                 "samples": len(self.samples)}
+
+
+_T0 = time.time()
+
+
+def log(msg: str) -> None:
+    """Progress on stderr (the JSON line alone goes to stdout)."""
+    sys.stderr.write(f"[bench {time.time() - _T0:7.1f}s] {msg}\n")
+    sys.stderr.flush()
 
 
 def reduce_max(x: float, device=None) -> float:
@@ -284,6 +349,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the long-context and packed-batch objects")
+    ap.add_argument("--extra-launches", type=int, default=4)
     ap.add_argument("--backward-calls", type=int, default=5)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -313,29 +381,55 @@ def main():
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, dev)
 
-    hbm_peak, _, peak_src = load_peaks()
+    hbm_peak, tc_peak, peak_src = load_peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # twice the 126 MB L2
+
+    def upload(inp):
+        tdt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+        host = {k: torch.from_numpy(getattr(inp, k)).to(tdt if k != "log_alpha" else torch.float32)
+                for k in ("q", "k", "v", "b", "w", "log_alpha")}
+        t = {k: x.to(dev) for k, x in host.items()}
+        t["s0"] = torch.from_numpy(inp.init_state).to(dev) if inp.init_state is not None else None
+        t["cu"] = (torch.from_numpy(inp.cu_seqlens.astype(np.int32)).to(dev)
+                   if inp.cu_seqlens is not None else None)
+        B, T, H, d = inp.q.shape
+        t["o"] = torch.empty((B, T, H, d), dtype=tdt, device=dev)
+        t["sf"] = torch.empty((inp.num_seqs, H, d, d), dtype=torch.float32, device=dev)
+        code = gdr2.GDR2_BF16 if inp.dtype == "bf16" else gdr2.GDR2_FP32
+        wsb = gdr2.workspace_size(B, T, H, d, d, inp.num_seqs, code)
+        t["ws"] = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+        t["ws_bytes"] = wsb
+        return host, t
+
+    def fwd(t):
+        gdr2.chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], t["s0"], t["cu"],
+                       o=t["o"], final_state=t["sf"], workspace=t["ws"])
+
+    def per_launch(fn, n, flush=False):
+        """Per-launch CUDA-event times (ms) of n launches of fn, each bracketed
+        by its own events; with flush, a 256 MiB write precedes every launch
+        (outside the events)."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in ev:
+            if flush:
+                flush_buf.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    log(f"generating the {args.workload} workload")
     inp, label = workload(args.workload)
-    tdt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
-    host = {k: torch.from_numpy(getattr(inp, k)).to(tdt if k != "log_alpha" else torch.float32)
-            for k in ("q", "k", "v", "b", "w", "log_alpha")}
-    dv_ = {k: x.to(dev) for k, x in host.items()}
-    s0 = torch.from_numpy(inp.init_state).to(dev) if inp.init_state is not None else None
-    cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).to(dev) if inp.cu_seqlens is not None else None
+    host, t = upload(inp)
+    log("timing the chunk forward")
     N = inp.num_seqs
     B, T, H, d = inp.q.shape
-    o = torch.empty((B, T, H, d), dtype=tdt, device=dev)
-    sf = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
-    dcode = gdr2.GDR2_BF16 if inp.dtype == "bf16" else gdr2.GDR2_FP32
-    ws_bytes = gdr2.workspace_size(B, T, H, d, d, N, dcode)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-
-    def step():
-        gdr2.chunk_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["log_alpha"], dv_["b"], dv_["w"], s0, cu,
-                       o=o, final_state=sf, workspace=ws)
-
+    step = lambda: fwd(t)
     # the chunk kernel; plus the order kernel of a packed batch, or the combine
     # and correction kernels of a segment split (few long sequences)
-    launches_per_step = 1 + (1 if cu is not None and N > 1 else 0) + (2 if cu is None and ws_bytes > 0 else 0)
+    launches_per_step = (1 + (1 if t["cu"] is not None and N > 1 else 0)
+                         + (2 if t["cu"] is None and t["ws_bytes"] > 0 else 0))
     clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     with clocks:
         for _ in range(args.warmup):
@@ -348,21 +442,48 @@ def main():
             ev[i + 1].record(stream)
         barrier()
         per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-        total_ms = ev[0].elapsed_time(ev[-1])
-        total_ms = max_over_ranks(total_ms)
+        total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]))
+        flushed = per_launch(step, min(args.steps, 20), flush=True)
+        barrier()
+        log(f"chunk forward: {1e3 * statistics.median(per):.1f} us median")
 
-        # Decode: 64 consecutive single-token steps on N=256 x H=16 heads.
-        dec = gen.decode_batch(steps=4)
+        # The other chunk-forward workloads, a few launches each.
+        extra = {}
+        if not args.no_extra_workloads:
+            for name in ("long", "varlen"):
+                if name == args.workload:
+                    continue
+                log(f"generating the {name} workload")
+                x_inp, x_label = workload(name)
+                _, xt = upload(x_inp)
+                log(f"timing {name}")
+                xstep = lambda xt=xt: fwd(xt)
+                xstep()
+                barrier()
+                xper = per_launch(xstep, args.extra_launches)
+                st = stats_ms(xper)
+                roof = chunk_roofline(x_inp, st["median_us"], hbm_peak, tc_peak, peak_src)
+                extra[name] = {"workload": x_label, "tokens": x_inp.num_tokens, "launches": len(xper),
+                               **st, "roofline": roof,
+                               "segments": ("split" if xt["cu"] is None and xt["ws_bytes"] > 0 else "serial"),
+                               "tokens_per_s": x_inp.num_tokens / (st["median_us"] * 1e-6)}
+                del xt
+                torch.cuda.empty_cache()
+            barrier()
+
+        # Decode: consecutive single-token steps on N=256 x H=16 heads, fresh
+        # token inputs every step.
+        log("decode")
+        dec = gen.decode_batch(steps=args.decode_steps)
         Nd, Hd, dkd = dec.q.shape[1:]
         dvd = dec.v.shape[-1]
         dstate = torch.from_numpy(dec.state).to(dev)
-        dtok = [{k: torch.from_numpy(getattr(dec, k)[i]).to(dev, torch.bfloat16 if k != "log_alpha"
-                                                            else torch.float32)
-                 for k in ("q", "k", "v", "b", "w", "log_alpha")} for i in range(4)]
+        dtok = {k: torch.from_numpy(getattr(dec, k)).to(dev, torch.bfloat16 if k != "log_alpha" else torch.float32)
+                for k in ("q", "k", "v", "b", "w", "log_alpha")}
         do = torch.empty((Nd, Hd, dvd), dtype=torch.bfloat16, device=dev)
 
         def dstep(i):
-            x = dtok[i % 4]
+            x = {k: v[i % args.decode_steps] for k, v in dtok.items()}
             gdr2.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], dstate, o=do)
 
         for i in range(3):
@@ -379,17 +500,18 @@ def main():
         # End to end: pinned host inputs in, o and final states out, every step.
         e2e = None
         if not args.no_e2e:
+            log("end to end")
             pinned = {k: x.pin_memory() for k, x in host.items()}
-            o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-            sf_h = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+            o_h = torch.empty(t["o"].shape, dtype=t["o"].dtype).pin_memory()
+            sf_h = torch.empty(t["sf"].shape, dtype=t["sf"].dtype).pin_memory()
             e2e_steps = max(3, min(args.steps, 20))
 
             def e2e_step():
                 for k in pinned:
-                    dv_[k].copy_(pinned[k], non_blocking=True)
+                    t[k].copy_(pinned[k], non_blocking=True)
                 step()
-                o_h.copy_(o, non_blocking=True)
-                sf_h.copy_(sf, non_blocking=True)
+                o_h.copy_(t["o"], non_blocking=True)
+                sf_h.copy_(t["sf"], non_blocking=True)
 
             for _ in range(2):
                 e2e_step()
@@ -402,7 +524,7 @@ def main():
             barrier()
             e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
             h2d = sum(x.numel() * x.element_size() for x in pinned.values())
-            d2h = o.numel() * o.element_size() + sf.numel() * sf.element_size()
+            d2h = t["o"].numel() * t["o"].element_size() + t["sf"].numel() * t["sf"].element_size()
             e2e = {"value": aggregate_throughput(inp.num_tokens, world, e2e_ms), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "ms_per_step": e2e_ms}
@@ -410,42 +532,42 @@ def main():
         # Backward on the same batch (after everything above: it reuses o's dtype for d_o).
         bwd = None
         if not args.no_backward:
+            log("backward")
             gen_do, gen_df = gen.cotangents(inp, seed=7)
-            d_o = torch.from_numpy(gen_do).to(dev, tdt)
+            d_o = torch.from_numpy(gen_do).to(dev, t["o"].dtype)
             d_fin = torch.from_numpy(gen_df).to(dev)
+            dcode = gdr2.GDR2_BF16 if inp.dtype == "bf16" else gdr2.GDR2_FP32
             bws = torch.empty(gdr2.bwd_workspace_size(B, T, H, d, d, N, dcode), dtype=torch.uint8,
                               device=dev)
 
             def bstep():
-                return gdr2.chunk_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["log_alpha"], dv_["b"],
-                                      dv_["w"], d_o, s0, d_fin, cu, workspace=bws)
+                return gdr2.chunk_bwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], d_o,
+                                      t["s0"], d_fin, t["cu"], workspace=bws)
 
             for _ in range(3):
                 bstep()
             barrier()
-            bev = [torch.cuda.Event(enable_timing=True) for _ in range(args.backward_calls + 1)]
-            bev[0].record(stream)
-            for i in range(args.backward_calls):
-                bstep()
-                bev[i + 1].record(stream)
-            barrier()
-            bper = [bev[i].elapsed_time(bev[i + 1]) for i in range(args.backward_calls)]
-            bms = max_over_ranks(statistics.mean(bper))
+            bper = per_launch(bstep, args.backward_calls)
+            bst = stats_ms(bper)
+            bms = max_over_ranks(bst["mean_us"]) * 1e-3
             fl = bwd_flops(inp)
             bwd = {"kernels": "column sweeps + per-chunk rows (2 launches)", "calls": args.backward_calls,
-                   "us_per_call": bms * 1e3, "tokens_per_s": inp.num_tokens / (bms * 1e-3),
+                   **bst, "us_per_call": bms * 1e3, "tokens_per_s": inp.num_tokens / (bms * 1e-3),
                    "bound": "alu", "flops_per_call": fl, "achieved_tflops": fl / (bms * 1e-3) / 1e12,
                    "peak_tflops": SIMT_FP32_TFLOPS, "frac": fl / (bms * 1e-3) / 1e12 / SIMT_FP32_TFLOPS,
                    "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz"}
 
     ms_per_step = total_ms / args.steps
     value = aggregate_throughput(inp.num_tokens, world, ms_per_step)
-    kern_ms = statistics.mean(per)
-    nbytes = chunk_bytes(inp)
-    achieved = nbytes / (kern_ms * 1e-3) / 1e9
+    pst = stats_ms(per)
+    fst = stats_ms(flushed)
+    roof = chunk_roofline(inp, pst["median_us"], hbm_peak, tc_peak, peak_src)
+    roof.update({"traffic": measured_traffic() if args.workload == "prefill" else None,
+                 "kernel": "chunk forward (chunk_tc_kernel)", "us_per_launch": pst["median_us"], **pst,
+                 "time_used": "median of the back-to-back launches"})
     dbytes = decode_bytes(Nd, Hd, dkd, dvd)
-    dmean = statistics.mean(dper)
-    dgbs = dbytes / (dmean * 1e-3) / 1e9
+    dst = stats_ms(dper)
+    dgbs = dbytes / (dst["median_us"] * 1e-6) / 1e9
 
     if rank != 0:
         if world > 1:
@@ -461,24 +583,26 @@ def main():
         "config": {"workload": label, "global_batch": world * B, "seq_len": T, "heads": H,
                    "d_k": d, "d_v": d, "tokens_per_rank": inp.num_tokens,
                    "parallelism": f"replicas x{world} (independent sequences per GPU)",
-                   "l2": "inputs larger than L2 (no flush)"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak,
-                     "traffic": measured_traffic() if args.workload == "prefill" else None,
-                     "kernel": "chunk forward", "bytes_per_launch": nbytes,
-                     "us_per_launch": kern_ms * 1e3, "peak_source": peak_src},
-        "decode": {"workload": "N=256 x H=16, d=128, fp32 state, bf16 tokens",
-                   "steps": args.decode_steps, "us_per_step": dmean * 1e3,
+                   "l2": "inputs larger than L2 (no flush between the timed steps); "
+                         "l2_flushed repeats the launch after a 256 MiB write"},
+        "roofline": roof,
+        "l2_flushed": {"launches": len(flushed), **fst,
+                       "frac": chunk_roofline(inp, fst["median_us"], hbm_peak, tc_peak, peak_src)["frac"]},
+        "decode": {"workload": "N=256 x H=16, d=128, fp32 state, bf16 tokens (fresh every step)",
+                   "steps": args.decode_steps, "us_per_step": dst["median_us"], **dst,
                    "bytes_per_step": dbytes, "achieved_gbs": dgbs, "peak_gbs": hbm_peak,
-                   "frac": dgbs / hbm_peak, "peak_source": peak_src},
+                   "frac": dgbs / hbm_peak, "peak_source": peak_src,
+                   "time_used": "median step"},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks.summary(),
     }
+    line.update(extra)
     if e2e is not None:
         line["e2e"] = e2e
     if bwd is not None:
         line["backward"] = bwd
     if world == 1 and not args.no_cpu_baseline:
+        log("cpu baseline")
         line["cpu_baseline"] = cpu_baseline(inp, label)
         if bwd is not None:
             bwd["cpu_baseline"] = cpu_backward_baseline(inp, gen_do, label)

@@ -44,9 +44,14 @@
  *     synchronisation, as for any CUDA kernel.
  *   - `o` may not alias any input. Calls that share output or state buffers
  *     must be ordered by the caller (same stream or events).
- *   - Decay range: within one 64-token chunk the summed log_alpha of any key
- *     channel must stay above -80 (per-token alpha above ~0.29 on average);
- *     below that the chunk form's fp32 decay factors leave the fp32 range.
+ *   - Decay: any alpha in (0, 1] (log_alpha <= 0, any magnitude). The chunk
+ *     kernels use the chunk form while the cumulative log-decay of every key
+ *     channel stays within 64 of its value at the chunk's middle row (decay
+ *     factors e^{+-64}); a chunk past that (a channel forgetting faster than
+ *     about e^-2 per token on average) is computed on the device by the exact
+ *     token recurrence instead -- for the bf16 d = 128 kernel the whole
+ *     (sequence, head) unit, otherwise that chunk -- which is slower but
+ *     exact to fp32 rounding. Nothing is reported and nothing is clamped.
  */
 #ifndef GDR2_H_
 #define GDR2_H_
@@ -168,7 +173,10 @@ gdr2_status gdr2_chunk_fwd_workspace_size(int64_t B, int64_t T, int64_t H,
  *     the serial scan, never the segment-parallel one).
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture. The address is kept for the rest of the process, so the
+ *     calls must run in the device's primary context (the CUDA runtime's
+ *     default) and not after a cudaDeviceReset; a lookup that fails returns
+ *     GDR2_ERR_CUDA and is tried again on the next call.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents; each call rewrites every entry it reads, so nothing has to be
  *     cleared, but calls that overlap on the GPU (unordered streams) race on

@@ -287,14 +287,22 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None
     `final_state`, if wanted) must be preallocated; nothing is allocated here."""
     import torch
     dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("chunk_fwd_noalloc needs CUDA tensors")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
     code = _dtype_code(q)
     for name, t, d in (("k", k, dk), ("b", b, dk), ("v", v, dv), ("w", w, dv)):
         _check(t, name, (B, T, H, d), dt, dev)
+    _check(q, "q", (B, T, H, dk), dt, dev)
     _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
-    N = cu_seqlens.shape[0] - 1 if cu_seqlens is not None else B
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+        N = cu_seqlens.shape[0] - 1
+    else:
+        N = B
     _check(o, "o", (B, T, H, dv), dt, dev)
     if init_state is not None:
         _check(init_state, "init_state", (N, H, dk, dv), torch.float32, dev)

@@ -527,8 +527,7 @@ cudaError_t launch_typed(const BwdParams &p, int64_t slots, cudaStream_t stream)
     }
     if (p.tokens > 0) {
         constexpr size_t smem = rows_smem_bytes<Tin, D>();
-        cudaError_t e = cudaFuncSetAttribute(bwd_rows_kernel<Tin, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_dynamic_smem((const void *)bwd_rows_kernel<Tin, D>, (int)smem);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)slots, (unsigned)p.H);
         bwd_rows_kernel<Tin, D><<<grid, kRowThreads, smem, stream>>>(p);

@@ -19,7 +19,9 @@
 // Range: the products ebar_r . kbar_s and qbar_r . kbar_s only need
 // e^{g_r - g_s} <= 1, so they are formed about the chunk's middle row m
 // (factors e^{+-(g - g_m)}), which halves the exponent range; the state-side
-// products use e^{g_r} <= 1 directly.
+// products use e^{g_r} <= 1 directly. A chunk in which |g_r - g_m| passes
+// kFactorRange on some channel (decay too strong for those factors) runs
+// the token rule itself instead, one token at a time, exact for any alpha.
 //
 // One CTA owns one (sequence, head, 32-wide value tile) and walks its chunks
 // in order, keeping the fp32 state tile in shared memory.
@@ -33,6 +35,9 @@ constexpr int kThreads = 256;
 constexpr int kDVT = 32;          // value columns per CTA
 constexpr int kLD = kChunk + 4;   // padded row length of [channel][row] arrays
 constexpr int kMid = 31;          // reference row for the pairwise products
+// Largest |g_r - g_m| (natural log) the factors e^{+-(g_r - g_m)} may take:
+// e^64 and e^-64 are normal fp32 numbers with room for the products they enter.
+constexpr float kFactorRange = 64.f;
 
 template <int DK>
 struct SimtSmem {
@@ -44,8 +49,10 @@ struct SimtSmem {
     float s0[DK][kDVT];    // state tile (fp32 master)
     float sm[DK][kDVT];    // Diag(e^{g_m}) S0
     float z[kChunk][kDVT]; // z -> r = z - Ebar S0 -> u (in place)
+    float la[DK][kLD];     // log alpha of the chunk (used by a token-serial chunk)
     float gC[DK];
     float gm[DK];
+    int serial;            // this chunk runs token by token
     float qinv[kChunk];    // prologue: 1 / ||q_r||, 1 / ||k_r|| (1 without it)
     float kinv[kChunk];
 };
@@ -72,8 +79,7 @@ chunk_simt_kernel(ChunkArgs args)
 
     int64_t t_begin, t_end;
     if (args.cu_seqlens) {
-        t_begin = args.cu_seqlens[n];
-        t_end = args.cu_seqlens[n + 1];
+        packed_bounds(args.cu_seqlens, n, args.B * args.T, t_begin, t_end);
     } else {
         t_begin = n * args.T;
         t_end = t_begin + args.T;
@@ -85,6 +91,7 @@ chunk_simt_kernel(ChunkArgs args)
         sm.s0[c][j] = args.init_state ? args.init_state[state_off + (int64_t)c * DV + j] : 0.f;
     }
 
+    if (tid == 0) sm.serial = 0;
     const uint32_t pre = kPre ? args.pre : 0u;
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kChunk) {
         const int L = (int)(t_end - t0 < kChunk ? t_end - t0 : kChunk);
@@ -117,17 +124,27 @@ chunk_simt_kernel(ChunkArgs args)
         if constexpr (kPre) __syncthreads();
 
         // ---- cumulative log-decay and decay-absorbed factors -------------
+        float g[kChunk];
         if (tid < DK) {
             const int c = tid;
-            float g[kChunk];
             float acc = 0.f;
 #pragma unroll
             for (int r = 0; r < kChunk; ++r) {
                 float x = r < L ? la[((t0 + r) * H + h) * DK + c] : 0.f;
                 if ((pre & GDR2_PROLOGUE_DECAY_SOFTPLUS) && r < L) x = pre_neg_softplus(x);
+                sm.la[c][r] = x;
                 acc += x;
                 g[r] = acc;
             }
+            float m = 0.f;
+#pragma unroll
+            for (int r = 0; r < kChunk; ++r) m = fmaxf(m, fabsf(g[r] - g[kMid]));
+            if (m > kFactorRange) sm.serial = 1;
+        }
+        __syncthreads();
+        const bool serial = sm.serial != 0;
+        if (tid < DK) {
+            const int c = tid;
             const float gm = g[kMid];
             sm.gC[c] = g[kChunk - 1];
             sm.gm[c] = gm;
@@ -145,7 +162,8 @@ chunk_simt_kernel(ChunkArgs args)
                     bv = to_f32(b[i]);
                     if (pre & GDR2_PROLOGUE_GATE_SIGMOID) bv = pre_sigmoid(bv);
                 }
-                const float up = expf(g[r] - gm), dn = expf(gm - g[r]);
+                // (a token-serial chunk keeps the raw q, k and b . k)
+                const float up = serial ? 1.f : expf(g[r] - gm), dn = serial ? 1.f : expf(gm - g[r]);
                 sm.qm[c][r] = qv * up;
                 sm.km[c][r] = kv * dn;
                 sm.em[c][r] = bv * kv * up;
@@ -163,6 +181,54 @@ chunk_simt_kernel(ChunkArgs args)
             sm.z[r][j] = zv;
         }
         __syncthreads();
+
+        if (serial) {
+            // ---- the token rule, one token at a time (decay past the factor
+            // range): s' = alpha . s, r = e^T s', s = s' + k (z - r),
+            // o = q^T s = q^T s' + (k^T q)(z - r). Thread (jc, rg) holds key
+            // channels rg * CPT .. + CPT - 1 of value column jc.
+            constexpr int CPT = DK / (kThreads / kDVT);
+            const int jc = tid % kDVT, rg = tid / kDVT, cb = rg * CPT;
+            float *red = &sm.a[0][0];  // [2][2][8][32] partial sums, then [2][8] k^T q
+            float *kqp = red + 2 * 2 * 8 * kDVT;
+            float st[CPT];
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) st[i] = sm.s0[cb + i][jc];
+            int buf = 0;
+            for (int r = 0; r < L; ++r) {
+                float pe = 0.f, pq = 0.f, pkq = 0.f;
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int c = cb + i;
+                    st[i] *= expf(sm.la[c][r]);
+                    pe = fmaf(sm.em[c][r], st[i], pe);
+                    pq = fmaf(sm.qm[c][r], st[i], pq);
+                    pkq = fmaf(sm.km[c][r], sm.qm[c][r], pkq);
+                }
+                float *rb = red + buf * 2 * 8 * kDVT;
+                rb[rg * kDVT + jc] = pe;
+                rb[8 * kDVT + rg * kDVT + jc] = pq;
+                if (jc == 0) kqp[buf * 8 + rg] = pkq;
+                __syncthreads();
+                float rr = 0.f, pp = 0.f, kq = 0.f;
+#pragma unroll
+                for (int gi = 0; gi < 8; ++gi) {
+                    rr += rb[gi * kDVT + jc];
+                    pp += rb[8 * kDVT + gi * kDVT + jc];
+                    kq += kqp[buf * 8 + gi];
+                }
+                const float delta = sm.z[r][jc] - rr;
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) st[i] = fmaf(sm.km[cb + i][r], delta, st[i]);
+                if (rg == 0) o[((t0 + r) * H + h) * DV + j0 + jc] = from_f32<Tin>(fmaf(kq, delta, pp));
+                buf ^= 1;
+            }
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) sm.s0[cb + i][jc] = st[i];
+            __syncthreads();
+            if (tid == 0) sm.serial = 0;  // (read again only after the next chunk's first barrier)
+            continue;
+        }
 
         // ---- A = strict_tril(Ebar Kbar^T), P = tril(Qbar Kbar^T) ----------
         {
@@ -282,7 +348,7 @@ cudaError_t launch_t(const ChunkArgs &a, cudaStream_t stream)
 {
     const size_t smem = sizeof(SimtSmem<DK>);
     auto kern = a.pre ? chunk_simt_kernel<Tin, DK, true> : chunk_simt_kernel<Tin, DK, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(a.dv / kDVT), (unsigned)a.H, (unsigned)a.num_seqs);
     kern<<<grid, kThreads, smem, stream>>>(a);

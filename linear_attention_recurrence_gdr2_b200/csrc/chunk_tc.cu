@@ -62,28 +62,6 @@ namespace gdr2 {
 
 __device__ int g_chunk_tc_error;
 
-// Optional per-phase SM-clock timestamps for CTAs 0-3 and 20-23 (compiled in
-// only with -DGDR2_TRACE; the tracing driver points g_chunk_tc_trace at a
-// buffer of [8 CTAs][1024 chunks][32 events] uint64).
-#ifdef GDR2_TRACE
-__device__ unsigned long long *g_chunk_tc_trace;
-#define GDR2_TRACE_AT(chunk, ev)                                                                \
-    do {                                                                                        \
-        const unsigned ts_ = blockIdx.x < 4 ? blockIdx.x : (blockIdx.x - 20u < 4u ? blockIdx.x - 16u : 8u); \
-        if (ts_ < 8 && g_chunk_tc_trace && (chunk) < 1024)                                      \
-            g_chunk_tc_trace[((size_t)ts_ * 1024 + (chunk)) * 32 + (ev)] = clock64();           \
-    } while (0)
-// [CTA][start ns, end ns, SM id] for every CTA (buffer sized by the driver)
-__device__ unsigned long long *g_chunk_tc_span;
-#define GDR2_SPAN_AT(slot, value)                                                          \
-    do {                                                                                   \
-        if (g_chunk_tc_span) g_chunk_tc_span[(size_t)blockIdx.x * 3 + (slot)] = (value);   \
-    } while (0)
-#else
-#define GDR2_TRACE_AT(chunk, ev) do { } while (0)
-#define GDR2_SPAN_AT(slot, value) do { } while (0)
-#endif
-
 namespace {
 
 using namespace sm100;
@@ -92,6 +70,14 @@ constexpr int kD = 128;
 constexpr int kThreadsTC = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;  // one second per wait
 constexpr int kPairs = 2;                     // (sequence, head) units per cluster
+// Largest |g_r - g_31| (natural log) the chunk form's factors e^{+-(g_r - g_31)}
+// may take: e^64 and e^-64 are normal fp32 / bf16 numbers with room for the
+// products and sums they enter.
+constexpr float kFactorRange = 64.f;
+// Largest decay (natural log) over the 64 tokens from one chunk's middle row
+// to the next one's: the epilogue moves the state between those two frames
+// with the single factor e^{-that}, which must stay a normal fp32 number.
+constexpr float kWindowRange = 80.f;
 
 // ---- main CTA shared memory (bytes from the 1024-aligned base) -------------
 __host__ __device__ constexpr uint32_t mEQ(int s) { return s ? 32768 : 0; }          // per key block kb: [Em -> -W 8K | Qm 8K]
@@ -118,7 +104,8 @@ constexpr uint32_t kH_BSUM = hVEC(1) + 1024;     // per-row-block log-decay sums
 // ---- both ------------------------------------------------------------------
 constexpr uint32_t kBAR = kH_BSUM + 8 * 128 * 4;   // same offset in both CTAs
 constexpr int kNumBars = 32;
-constexpr uint32_t kMISC = kBAR + kNumBars * 8;    // TMEM slot, abort flag, copy counters
+constexpr uint32_t kMISC = kBAR + kNumBars * 8;    // TMEM slot, abort flag, copy counters, range flag
+constexpr uint32_t kRangeFlagOff = 32;             // (within kMISC)
 constexpr uint32_t kSmemBytes = kMISC + 64 + 1024; // + alignment slack
 static_assert(kM_OST + 64 * kOPitch <= kM_WT && kM_WT + 16384 <= kBAR,
               "main shared-memory map overlaps the barriers");
@@ -158,6 +145,7 @@ constexpr uint32_t kBarZ = 1, kBarEpi = 2, kBarW = 3;   // main
 constexpr uint32_t kBarPrepA = 1, kBarPrepB = 3;        // helper
 
 struct TcParams {
+    const __nv_bfloat16 *q, *k, *b, *v;  // (read directly only by the serial path)
     const float *la;
     const __nv_bfloat16 *w;
     const float *init_state;
@@ -166,6 +154,7 @@ struct TcParams {
     __nv_bfloat16 *o;
     float *final_state;
     int64_t T, H, units;
+    int64_t tokens;  // B * T: every token range lies inside [0, tokens)
     // segment-parallel scan (nseg > 1): per sequence, jobs 0..nseg-1 run the
     // segments from their entry state (the true one for segment 0, else 0) and
     // write o and seg_s0; jobs nseg..2 nseg-2 run segments 1..nseg-1 from the
@@ -301,6 +290,202 @@ __device__ __forceinline__ void store_row_bf16_sw128(unsigned char *tile, uint32
 __device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory"); }
 __device__ __forceinline__ void setmaxnreg_inc152() { asm volatile("setmaxnreg.inc.sync.aligned.u32 152;" ::: "memory"); }
 
+// The work of one CTA pair: its (sequence, head) unit, token range and
+// states. Unit u = (cluster, position in it); with a segment split, each
+// (sequence, head) has 2 nseg - 1 jobs: segments 0..nseg-1 from their entry
+// state (the true one for segment 0, else zero), then segments 1..nseg-1 from
+// the identity with z = 0.
+struct UnitJob {
+    bool valid;             // false for the padding pair of the last cluster
+    bool zero_v;            // identity-state run with z = 0 (writes psi and Phi)
+    int64_t h, t_begin, t_end;
+    const float *init_ptr;  // entry state, or null (zero, or the identity if zero_v)
+    float *final_ptr;       // where the exit state goes, or null
+};
+
+__device__ __forceinline__ UnitJob unit_job(const TcParams &prm, uint32_t cta, uint32_t rank)
+{
+    UnitJob u{false, false, 0, 0, 0, nullptr, nullptr};
+    const int64_t H = prm.H;
+    const int64_t unit = (int64_t)(cta / (2 * kPairs)) * kPairs + (rank % kPairs);
+    if (unit >= prm.units) return u;
+    u.valid = true;
+    const int jobs = 2 * prm.nseg - 1;
+    const int64_t nj = unit / H;
+    u.h = unit % H;
+    const int job = (int)(nj % jobs);
+    const int64_t n = prm.order ? (int64_t)prm.order[nj / jobs] : (int64_t)(nj / jobs);
+    if (prm.cu_seqlens) {
+        packed_bounds(prm.cu_seqlens, n, prm.tokens, u.t_begin, u.t_end);
+    } else {
+        u.t_begin = n * prm.T;
+        u.t_end = u.t_begin + prm.T;
+    }
+    u.zero_v = job >= prm.nseg;
+    const int seg = u.zero_v ? job - prm.nseg + 1 : job;
+    if (prm.nseg > 1) {
+        const int64_t sb = u.t_begin + seg * prm.seg_len;
+        u.t_end = sb + prm.seg_len < u.t_end ? sb + prm.seg_len : u.t_end;
+        u.t_begin = sb;
+    }
+    const int64_t state_base = (n * H + u.h) * (int64_t)kD * kD;
+    if (prm.nseg == 1) {
+        u.init_ptr = prm.init_state ? prm.init_state + state_base : nullptr;
+        u.final_ptr = prm.final_state ? prm.final_state + state_base : nullptr;
+    } else {
+        const int64_t seg_base = ((n * prm.nseg + seg) * H + u.h) * (int64_t)kD * kD;
+        u.init_ptr = (!u.zero_v && seg == 0 && prm.init_state) ? prm.init_state + state_base : nullptr;
+        u.final_ptr = (u.zero_v ? prm.seg_phi : prm.seg_s0) + seg_base;
+    }
+    return u;
+}
+
+// Exact fp32 recurrence of one (sequence, head) unit, token by token, for the
+// value columns [j0, j0 + 64). A unit takes this path, after its chunk pass,
+// when some chunk's decay leaves the chunk form's factor range (kFactorRange):
+// it runs the token rule as the article states it ("Gated Delta Rule-2: two
+// gates instead of one", ainews.random.gg): decay, erase read e^T S', delta
+// write, readout with the post-update state, so any alpha in (0, 1] is exact
+// to fp32 rounding. Columns of S evolve independently of each other, so each
+// CTA of the pair takes half of them. All 512 threads: thread t holds key
+// channels 16 (t >> 6) .. +15 of column j0 + (t & 63) in registers (the code
+// runs after the role split, where the first warpgroup keeps 40 registers).
+constexpr int kSerTok = 16;  // tokens staged in shared memory per batch
+__device__ __forceinline__ void serial_unit(const TcParams &prm, const UnitJob &u, int j0,
+                                           unsigned char *smem, int t)
+{
+    const int64_t H = prm.H, h = u.h;
+    const bool zero_v = u.zero_v;
+    const int j = t & 63, kg = t >> 6, c0 = 16 * kg;
+    float *vec = reinterpret_cast<float *>(smem);  // [kSerTok][4][128]: alpha, e = b.k, k, q
+    float *zt = vec + kSerTok * 4 * kD;            // [kSerTok][64]: z = w.v of this CTA's columns
+    float *red = zt + kSerTok * 64;                // [2][2][8][64]: partial e^T S', q^T S'
+    float *kqp = red + 2 * 2 * 8 * 64;             // [2][8]: partial k^T q
+    float st[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i;
+        st[i] = u.init_ptr ? u.init_ptr[(int64_t)c * kD + j0 + j] : ((zero_v && c == j0 + j) ? 1.f : 0.f);
+    }
+    int buf = 0;
+    for (int64_t tb = u.t_begin; tb < u.t_end; tb += kSerTok) {
+        const int nb = (int)(u.t_end - tb < kSerTok ? u.t_end - tb : kSerTok);
+        __syncthreads();  // the previous batch has been consumed
+        {   // staging: token r = t >> 5, key channels 4 (t & 31) .. +3, two of z
+            const int r = t >> 5, cb = 4 * (t & 31);
+            float qf[4] = {0.f, 0.f, 0.f, 0.f}, kf[4] = {0.f, 0.f, 0.f, 0.f};
+            float bf[4] = {0.f, 0.f, 0.f, 0.f}, lf[4] = {0.f, 0.f, 0.f, 0.f};
+            if (r < nb) {
+                const int64_t base = ((tb + r) * H + h) * kD + cb;
+                const uint2 qr = *reinterpret_cast<const uint2 *>(prm.q + base);
+                const uint2 kr = *reinterpret_cast<const uint2 *>(prm.k + base);
+                const uint2 br = *reinterpret_cast<const uint2 *>(prm.b + base);
+                const float4 l4 = *reinterpret_cast<const float4 *>(prm.la + base);
+                float2 x = bf2_to_f2(qr.x), y = bf2_to_f2(qr.y);
+                qf[0] = x.x; qf[1] = x.y; qf[2] = y.x; qf[3] = y.y;
+                x = bf2_to_f2(kr.x); y = bf2_to_f2(kr.y);
+                kf[0] = x.x; kf[1] = x.y; kf[2] = y.x; kf[3] = y.y;
+                x = bf2_to_f2(br.x); y = bf2_to_f2(br.y);
+                bf[0] = x.x; bf[1] = x.y; bf[2] = y.x; bf[3] = y.y;
+                lf[0] = l4.x; lf[1] = l4.y; lf[2] = l4.z; lf[3] = l4.w;
+            }
+            if (prm.pre & GDR2_PROLOGUE_QK_L2NORM) {  // a warp holds one token's row
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    sq = fmaf(qf[i], qf[i], sq);
+                    sk = fmaf(kf[i], kf[i], sk);
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, m);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, m);
+                }
+                sq = rsqrtf(sq + 1e-6f);
+                sk = rsqrtf(sk + 1e-6f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    qf[i] *= sq;
+                    kf[i] *= sk;
+                }
+            }
+            if (r < nb) {
+                const bool sig = (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID) != 0;
+                const bool spl = (prm.pre & GDR2_PROLOGUE_DECAY_SOFTPLUS) != 0;
+                float *vr = vec + r * 4 * kD + cb;
+                float4 al, ev;
+                al.x = expf(spl ? pre_neg_softplus(lf[0]) : lf[0]);
+                al.y = expf(spl ? pre_neg_softplus(lf[1]) : lf[1]);
+                al.z = expf(spl ? pre_neg_softplus(lf[2]) : lf[2]);
+                al.w = expf(spl ? pre_neg_softplus(lf[3]) : lf[3]);
+                ev.x = (sig ? pre_sigmoid(bf[0]) : bf[0]) * kf[0];
+                ev.y = (sig ? pre_sigmoid(bf[1]) : bf[1]) * kf[1];
+                ev.z = (sig ? pre_sigmoid(bf[2]) : bf[2]) * kf[2];
+                ev.w = (sig ? pre_sigmoid(bf[3]) : bf[3]) * kf[3];
+                *reinterpret_cast<float4 *>(vr) = al;
+                *reinterpret_cast<float4 *>(vr + kD) = ev;
+                *reinterpret_cast<float4 *>(vr + 2 * kD) = make_float4(kf[0], kf[1], kf[2], kf[3]);
+                *reinterpret_cast<float4 *>(vr + 3 * kD) = make_float4(qf[0], qf[1], qf[2], qf[3]);
+                if (!zero_v) {
+                    const int cz = 2 * (t & 31);
+                    const int64_t vb = ((tb + r) * H + h) * kD + j0 + cz;
+                    const float2 vv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(prm.v + vb));
+                    float2 ww = bf2_to_f2(*reinterpret_cast<const uint32_t *>(prm.w + vb));
+                    if (sig) ww = make_float2(pre_sigmoid(ww.x), pre_sigmoid(ww.y));
+                    *reinterpret_cast<float2 *>(zt + r * 64 + cz) = make_float2(ww.x * vv.x, ww.y * vv.y);
+                }
+            }
+        }
+        __syncthreads();
+        for (int r = 0; r < nb; ++r) {
+            const float *vr = vec + r * 4 * kD + c0;
+            float pe = 0.f, pq = 0.f, pkq = 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const float4 a = *reinterpret_cast<const float4 *>(vr + 4 * i4);
+                st[4 * i4 + 0] *= a.x; st[4 * i4 + 1] *= a.y; st[4 * i4 + 2] *= a.z; st[4 * i4 + 3] *= a.w;
+                const float4 e = *reinterpret_cast<const float4 *>(vr + kD + 4 * i4);
+                pe = fmaf(e.x, st[4 * i4 + 0], pe); pe = fmaf(e.y, st[4 * i4 + 1], pe);
+                pe = fmaf(e.z, st[4 * i4 + 2], pe); pe = fmaf(e.w, st[4 * i4 + 3], pe);
+                const float4 q = *reinterpret_cast<const float4 *>(vr + 3 * kD + 4 * i4);
+                pq = fmaf(q.x, st[4 * i4 + 0], pq); pq = fmaf(q.y, st[4 * i4 + 1], pq);
+                pq = fmaf(q.z, st[4 * i4 + 2], pq); pq = fmaf(q.w, st[4 * i4 + 3], pq);
+                const float4 k = *reinterpret_cast<const float4 *>(vr + 2 * kD + 4 * i4);
+                pkq = fmaf(k.x, q.x, pkq); pkq = fmaf(k.y, q.y, pkq);
+                pkq = fmaf(k.z, q.z, pkq); pkq = fmaf(k.w, q.w, pkq);
+            }
+            float *rb = red + buf * 2 * 8 * 64;
+            rb[kg * 64 + j] = pe;
+            rb[8 * 64 + kg * 64 + j] = pq;
+            if (j == 0) kqp[buf * 8 + kg] = pkq;
+            __syncthreads();
+            float rr = 0.f, pp = 0.f, kq = 0.f;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                rr += rb[g * 64 + j];
+                pp += rb[8 * 64 + g * 64 + j];
+                kq += kqp[buf * 8 + g];
+            }
+            const float delta = (zero_v ? 0.f : zt[r * 64 + j]) - rr;
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const float4 k = *reinterpret_cast<const float4 *>(vr + 2 * kD + 4 * i4);
+                st[4 * i4 + 0] = fmaf(k.x, delta, st[4 * i4 + 0]);
+                st[4 * i4 + 1] = fmaf(k.y, delta, st[4 * i4 + 1]);
+                st[4 * i4 + 2] = fmaf(k.z, delta, st[4 * i4 + 2]);
+                st[4 * i4 + 3] = fmaf(k.w, delta, st[4 * i4 + 3]);
+            }
+            if (kg == 0)
+                (zero_v ? prm.psi : prm.o)[((tb + r) * H + h) * kD + j0 + j] = __float2bfloat16_rn(fmaf(kq, delta, pp));
+            buf ^= 1;
+        }
+    }
+    if (u.final_ptr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) u.final_ptr[(int64_t)(c0 + i) * kD + j0 + j] = st[i];
+    }
+}
+
 // kPre: the fused prologue is compiled in (only the *_preact calls launch it;
 // the plain kernel carries none of its code, which matters for instruction
 // fetch).
@@ -321,6 +506,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kMISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kMISC + 4);
     uint32_t *copy_count = reinterpret_cast<uint32_t *>(smem + kMISC + 8);  // helper: [F0 F1 P0 P1 T0 T1]
+    // set (in both CTAs of the pair) once a chunk's decay leaves the factors' range
+    volatile int *range_flag = reinterpret_cast<volatile int *>(smem + kMISC + kRangeFlagOff);
 
     // Cluster ranks [0, kPairs) are the main CTAs of kPairs units, ranks
     // [kPairs, 2 kPairs) their helpers (so that CTAs running the same code
@@ -331,45 +518,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     const uint32_t peer_abort = mapa_shared(sbase + kMISC + 4, peer);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = prm.H;
-    const int64_t unit = (int64_t)(blockIdx.x / (2 * kPairs)) * kPairs + (rank % kPairs);
-    const bool valid = unit < prm.units;  // the last cluster may hold a padding pair
-    const int jobs = 2 * prm.nseg - 1;    // per (sequence, head)
-    int64_t h = 0, n = 0, t_begin = 0, t_end = 0;
-    int job = 0;
-    if (valid) {
-        h = unit % H;
-        const int64_t nj = unit / H;
-        job = (int)(nj % jobs);
-        n = prm.order ? (int64_t)prm.order[nj / jobs] : (int64_t)(nj / jobs);
-        if (prm.cu_seqlens) {
-            t_begin = prm.cu_seqlens[n];
-            t_end = prm.cu_seqlens[n + 1];
-        } else {
-            t_begin = n * prm.T;
-            t_end = t_begin + prm.T;
-        }
-    }
-    // segment of this job, and whether it is an identity-state run with z = 0
-    const bool zero_v = job >= prm.nseg;
-    const int seg = zero_v ? job - prm.nseg + 1 : job;
-    if (prm.nseg > 1 && valid) {
-        const int64_t sb = t_begin + seg * prm.seg_len;
-        t_end = sb + prm.seg_len < t_end ? sb + prm.seg_len : t_end;
-        t_begin = sb;
-    }
+    const UnitJob job = unit_job(prm, blockIdx.x, rank);
+    const bool valid = job.valid;
+    const int64_t h = job.h, t_begin = job.t_begin, t_end = job.t_end;
+    const bool zero_v = job.zero_v;
+    const float *init_ptr = job.init_ptr;
+    float *final_ptr = job.final_ptr;
     const int nc = (int)((t_end - t_begin + 63) / 64);
-    const int64_t state_base = (n * H + h) * (int64_t)kD * kD;
-    // entry state (null: zero, unless identity) and where the exit state goes
-    const float *init_ptr = nullptr;
-    float *final_ptr = nullptr;
-    if (prm.nseg == 1) {
-        init_ptr = prm.init_state ? prm.init_state + state_base : nullptr;
-        final_ptr = prm.final_state ? prm.final_state + state_base : nullptr;
-    } else {
-        const int64_t seg_base = ((n * prm.nseg + seg) * H + h) * (int64_t)kD * kD;
-        init_ptr = (!zero_v && seg == 0 && prm.init_state) ? prm.init_state + state_base : nullptr;
-        final_ptr = (zero_v ? prm.seg_phi : prm.seg_s0) + seg_base;
-    }
 
     if (nc == 0) {
         // empty sequence (both CTAs of the pair are here): the final state is
@@ -394,6 +549,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             mbar_init(&bars[H_XFREE1], 2);
         }
         *abort_flag = 0;
+        *range_flag = 0;
         for (int i = 0; i < 6; ++i) copy_count[i] = 0;
         fence_mbar_init();
     }
@@ -413,13 +569,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     cluster_sync_all();  // barriers of both CTAs initialised before any remote access
     tc_fence_after();
     const uint32_t tb = *tmem_slot;
-    if (tid == 0) {
-        GDR2_TRACE_AT(0, 31);  // common time base of the two CTAs
-        uint32_t smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        GDR2_SPAN_AT(0, globaltimer_ns());
-        GDR2_SPAN_AT(2, smid);
-    }
 
     if (is_main) {
     // =========================================================================
@@ -439,7 +588,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     if (c >= 2 && !wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 1))
                         break;
                     const int z = (int)(t_begin + 64 * c);
-                    GDR2_TRACE_AT(c, 0);
                     mbar_arrive_expect_tx(&bars[M_VFULL0 + s], 16384);
                     for (int blk = 0; blk < 2; ++blk)
                         tma_load_3d(smem + mZ(s) + blk * 8192, &map_v, &bars[M_VFULL0 + s], 64 * blk, (int)h, z);
@@ -456,7 +604,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 if (c >= 2) {
                     if (!wait_bar(&bars[M_SLOTFREE0 + s], ((c >> 1) - 1) & 1, abort_flag, peer_abort, 2)) break;
                     mbar_remote_arrive(h_mfree + 8 * s);
-                    GDR2_TRACE_AT(c - 2, 15);
                 }
             }
             if (vissued0 > 0) drain_wait(&bars[M_VFULL0], (vissued0 - 1) & 1, 20);
@@ -482,7 +629,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 // the W columns once chunk c-1's -W has been read out
                 if (c >= 1 && !wait_bar(&bars[M_UCONV], (c - 1) & 1, abort_flag, peer_abort, 15)) break;
                 if (c >= 1 && !wait_bar(&bars[M_WFREE], (c - 1) & 1, abort_flag, peer_abort, 16)) break;
-                GDR2_TRACE_AT(c, 1);
                 tc_fence_after();
                 // -W rows r (M = 64, A negated): key channels of block kb -> lanes 16 kb .. 16 kb + 15
 #pragma unroll
@@ -496,7 +642,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     mma_ss(tb + kTmU, desc_at(dz, kk * 2048), desc_at(dt, kk * 32), i_u, kk > 0);
                 tc_commit(&bars[M_WDONE]);
                 tc_commit(&bars[M_VFREE0 + s]);
-                GDR2_TRACE_AT(c, 2);
             }
             tc_commit(&bars[M_DRAIN]);
             drain_wait(&bars[M_DRAIN], 0, 22);
@@ -510,7 +655,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const int s = c & 1;
                 if (!wait_bar(&bars[M_F0 + s], (c >> 1) & 1, abort_flag, peer_abort, 3)) break;
                 mbar_remote_arrive(h_slotfree + 8 * s);
-                GDR2_TRACE_AT(c, 3);
             }
         }
     } else {
@@ -525,7 +669,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const uint64_t dwq = desc_at(d_wq, mEQ(s) - mEQ(0)), dpk = desc_at(d_pk, mKB(s) - mKB(0));
                 if (!spin_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
                 if (!spin_bar(&bars[M_SREADY_LO], c & 1, abort_flag, peer_abort, 18)) break;
-                GDR2_TRACE_AT(c, 4);
                 tc_fence_after();
                 // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows); the
                 // state arrives in two halves of 64 key channels (K steps 0-3, 4-7)
@@ -538,10 +681,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 for (int kk = 4; kk < 8; ++kk)
                     mma_ts(tb + kTmU, tb + kTmSB + kk * 8, desc_at(dwq, 16384 + (kk & 3) * 32), i_uo, 1);
                 tc_commit(&bars[M_UDONE]);
-                GDR2_TRACE_AT(c, 5);
                 if (!spin_bar(&bars[M_UCONV], c & 1, abort_flag, peer_abort, 19)) break;
                 if (!spin_bar(&bars[M_P0 + s], (c >> 1) & 1, abort_flag, peer_abort, 25)) break;
-                GDR2_TRACE_AT(c, 6);
                 tc_fence_after();
                 // [O^T | M^T] += U^T [P^T | Km]   (N = 192, B MN-major: P^T atom, two Km atoms)
 #pragma unroll
@@ -549,7 +690,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     mma_ts(tb + kTmO, tb + kTmUB + kk * 8, desc_at(dpk, kk * 2048), i_os, 1);
                 tc_commit(&bars[M_SDONE]);
                 tc_commit(&bars[M_SLOTFREE0 + s]);
-                GDR2_TRACE_AT(c, 7);
             }
             tc_commit(&bars[M_DRAIN2]);
             drain_wait(&bars[M_DRAIN2], 0, 23);
@@ -608,7 +748,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             fence_proxy_async_smem();
             named_bar_sync(kBarZ, 128);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 8);
                 mbar_arrive(&bars[M_ZREADY0 + s]);
                 mbar_arrive(&bars[M_WTFREE]);
             }
@@ -647,7 +786,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             // the W and U0 MMAs have read T: the helper may send chunk c + 2's T
             // (only chunks the helper still sends wait for this)
             if (tp == 0 && c + 2 < nc) mbar_remote_arrive(h_tfree + 8 * s);
-            GDR2_TRACE_AT(c, 9);
             tc_fence_after();
             uint32_t v0[32], v1[32];
             const uint32_t taddr = tb + kTmW + ((uint32_t)(32 * pw) << 16);
@@ -665,7 +803,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             fence_proxy_async_smem();
             named_bar_sync(kBarW, 128);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 10);
                 mbar_arrive(&bars[M_WFREE]);
                 mbar_arrive(&bars[M_WREADY0 + s]);
             }
@@ -732,7 +869,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             vecF[j] = expf(t1c + (last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j]));
             // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_UDONE], c & 1, abort_flag, peer_abort, 10))) break;
-            if (te == 0) GDR2_TRACE_AT(c, 11);
             tc_fence_after();
             {
                 uint32_t v0[32], v1[32], ub[16];
@@ -752,12 +888,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tc_fence_before();
             named_bar_sync(kBarEpi, 128);
             if (te == 0) {
-                GDR2_TRACE_AT(c, 12);
                 mbar_arrive(&bars[M_UCONV]);
             }
 
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_SDONE], c & 1, abort_flag, peer_abort, 11))) break;
-            if (te == 0) GDR2_TRACE_AT(c, 13);
             tc_fence_after();
             // O^T row j -> registers as bf16 pairs (rows r, r+1), then the O region
             // is zeroed for the next chunk; o is stored after the state hand-off
@@ -823,7 +957,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     }
                 }
             }
-            if (te == 0) GDR2_TRACE_AT(c, 14);
             // o rows of this chunk into the staging tile, from which the -W group
             // stores them to global memory; adjacent lanes (channels j, j+1) trade
             // halves so that the even lane writes rows 2q and the odd lane rows
@@ -865,7 +998,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     break;
                 const int z = (int)(t_begin + 64 * c);
                 unsigned char *eq = smem + hEQ(s), *kq = smem + hEQ(s) + kH_KmOff;
-                GDR2_TRACE_AT(c, 16);
                 mbar_arrive_expect_tx(&bars[H_FULL0 + s], 3 * 16384);
                 for (int blk = 0; blk < 2; ++blk) {
                     tma_load_3d(eq + blk * 16384, &map_b, &bars[H_FULL0 + s], 64 * blk, (int)h, z);
@@ -897,7 +1029,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                            desc_at(deq, (kk >> 2) * 16384 + (kk & 3) * 32), i_ap, kk > 0);
                 tc_commit(&bars[H_AP0 + s]);
                 tc_commit(&bars[H_SLOTFREE0 + s]);
-                GDR2_TRACE_AT(c, 17);
             }
             tc_commit(&bars[H_DRAIN]);
             drain_wait(&bars[H_DRAIN], 0, 22);
@@ -919,7 +1050,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 bulk_copy_to_cluster(rbase + mKB(s) + kKmOff, sbase + hEQ(s) + kH_KmOff, 16384, bar);
                 bulk_copy_to_cluster(rbase + mVEC(s), sbase + hVEC(s), 1024, bar);
                 copy_count[s] += 1;
-                GDR2_TRACE_AT(c, 23);
             }
         }
     }
@@ -939,6 +1069,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const float *la_s = reinterpret_cast<const float *>(smem + kH_LA);  // staged log_alpha [64][128]
         float *vecBS = reinterpret_cast<float *>(smem + kH_BSUM);          // [8][128]
         const uint32_t m_p = mapa_shared(smem_u32(&bars[M_P0]), peer);
+        const uint32_t peer_range_flag = mapa_shared(sbase + kMISC + kRangeFlagOff, peer);
         int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
         if (tp == 0) {
             ++la_issued;
@@ -955,7 +1086,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             unsigned char *k_tile = smem + hEQ(s) + kH_KmOff + kb * 8192;
 
             if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_LAFULL], c & 1, abort_flag, peer_abort, 3))) break;
-            if (tp == 0) GDR2_TRACE_AT(c, 18);
             float4 la[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -977,7 +1107,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (!group_and(kBarPrepA, 256, wait_bar(&bars[H_FULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 4)))
                 break;
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 19);
                 if (c + 1 < nc) {  // stage the next chunk's log_alpha
                     ++la_issued;
                     mbar_arrive_expect_tx(&bars[H_LAFULL], 32768);
@@ -998,6 +1127,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
                 if (pw == 0 || pw == 4)
                     *reinterpret_cast<float4 *>(smem + hVEC(s) + (pw == 0 ? 0 : 512) + 16 * g) = half;
+                // the state passes from chunk c-1's frame to chunk c's with the one factor
+                // e^{T1(c-1) + T0(c)} (second half of the last chunk, first half of this
+                // one), which has to stay a normal fp32 number
+                if (pw == 0 && c >= 1) {
+                    const float4 t1p = *reinterpret_cast<const float4 *>(smem + hVEC(s ^ 1) + 512 + 16 * g);
+                    const float a = fminf(fminf(t1p.x + half.x, t1p.y + half.y), fminf(t1p.z + half.z, t1p.w + half.w));
+                    if (a < -kWindowRange && !*range_flag) {
+                        *range_flag = 1;
+                        st_cluster_u32(peer_range_flag, 1u);
+                    }
+                }
                 if (pw < 4) {
 #pragma unroll
                     for (int i = 7; i >= 0; --i) {
@@ -1011,6 +1151,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         run.x += la[i].x; run.y += la[i].y; run.z += la[i].z; run.w += la[i].w;
                         la[i] = make_float4(run.x * kLog2e, run.y * kLog2e, run.z * kLog2e, run.w * kLog2e);
                     }
+                }
+            }
+            // range of the factors e^{+-d}: past it (decay of more than kFactorRange
+            // within half a chunk) the whole unit is recomputed exactly, token by
+            // token, once this pass is done (see serial_unit)
+            {
+                float m = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    m = fmaxf(m, fmaxf(fmaxf(fabsf(la[i].x), fabsf(la[i].y)), fmaxf(fabsf(la[i].z), fabsf(la[i].w))));
+                if (m > kFactorRange * kLog2e && !*range_flag) {
+                    *range_flag = 1;
+                    st_cluster_u32(peer_range_flag, 1u);
                 }
             }
             // prologue: 1 / ||q_r||, 1 / ||k_r|| (a warp holds whole rows: lanes
@@ -1081,7 +1234,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             fence_proxy_async_smem();
             named_bar_sync(kBarPrepA, 256);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 20);
                 mbar_arrive(&bars[H_FDONE]);  // to the MMA issuer and the factor sender
             }
             }  // c < nc
@@ -1098,7 +1250,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (!group_and(kBarPrepA, 256,
                            cp < 2 || wait_bar(&bars[H_MFREE0 + sp], ((cp >> 1) - 1) & 1, abort_flag, peer_abort, 7)))
                 break;
-            if (tp == 0) GDR2_TRACE_AT(cp, 21);
             tc_fence_after();
             {
                 const int q4 = pw & 3, hf = pw >> 2;
@@ -1127,7 +1278,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tc_fence_before();
             named_bar_sync(kBarPrepA, 256);
             if (tp == 0) {
-                GDR2_TRACE_AT(cp, 22);
                 mbar_arrive(&bars[H_XFREE0 + sp]);
                 if (!*abort_flag) {
                     const uint32_t bar = m_p + 8 * sp;
@@ -1150,7 +1300,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             const int s = c & 1;
             if (!group_and(kBarPrepB, 128, wait_bar(&bars[H_AP0 + s], (c >> 1) & 1, abort_flag, peer_abort, 8)))
                 break;
-            if (tp == 0) GDR2_TRACE_AT(c, 24);
             tc_fence_after();
             {   // A^T rows from the M=64 accumulator (lane i < 16 of warp pw: row s = 16 pw + i):
                 // A^T[s][r] = A[r][s] for r > s
@@ -1174,7 +1323,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             tc_fence_before();
             named_bar_sync(kBarPrepB, 128);
             if (tp == 0) {
-                GDR2_TRACE_AT(c, 25);
                 mbar_arrive(&bars[H_XFREE0 + s]);
             }
 
@@ -1214,7 +1362,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             named_bar_sync(kBarPrepB, 128);
-            if (tp == 0) GDR2_TRACE_AT(c, 26);
             {   // step 2a: Y = A_10 T_00 inside 32-block pb (warp: pb = pw >> 1, n-tile pw & 1)
                 const int pb = pw >> 1, nt = pw & 1, b0 = 32 * pb;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1252,7 +1399,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
             }
             named_bar_sync(kBarPrepB, 128);
-            if (tp == 0) GDR2_TRACE_AT(c, 27);
             // T into the bf16 buffer: its previous content (chunk c-2) has reached the
             // main CTA, and the main CTA's T buffer is free, once chunk c-2's W and U0
             // MMAs are done
@@ -1260,7 +1406,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                            c < 2 || wait_bar(&bars[H_TFREE0 + s], ((c >> 1) - 1) & 1, abort_flag,
                                                    peer_abort, 10)))
                 break;
-            if (tp == 0) GDR2_TRACE_AT(c, 28);
             {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
                 const int r = tp >> 1, half = tp & 1;
                 const float *trow = sT + r * kLD + 32 * half;
@@ -1284,7 +1429,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_remote_arrive_expect_tx(bar, 8192);
                 bulk_copy_to_cluster(mapa_shared(sbase + mT(s), peer), sbase + hT(s), 8192, bar);
                 copy_count[4 + s] += 1;
-                GDR2_TRACE_AT(c, 29);
             }
         }
     }
@@ -1307,8 +1451,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     }
     cluster_sync_all();
     tc_fence_after();
-    if (tid == 0) GDR2_SPAN_AT(1, globaltimer_ns());
     if (warp == 2) tmem_dealloc(tb, is_main ? 512 : 256);
+    // a chunk's decay left the factors' range: recompute the unit exactly (this
+    // CTA's half of the value columns; the chunk pass's o and state are replaced)
+    // (the job is derived again from fresh reads of the CTA's coordinates, so
+    // that none of the chunk pass's registers has to live until here)
+    if (*range_flag && !*abort_flag) {  // (the same decision in every thread of the CTA)
+        uint32_t cta;
+        asm volatile("mov.u32 %0, %%ctaid.x;" : "=r"(cta));
+        const uint32_t rk = cluster_ctarank();
+        serial_unit(prm, unit_job(prm, cta, rk), rk < (uint32_t)kPairs ? 0 : 64, smem, (int)threadIdx.x);
+    }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -1370,6 +1523,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
               make_map(&mw, a.w ? a.w : dummy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tk, a.H, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     TcParams p;
+    p.q = (const __nv_bfloat16 *)a.q;
+    p.k = (const __nv_bfloat16 *)a.k;
+    p.b = (const __nv_bfloat16 *)a.b;
+    p.v = (const __nv_bfloat16 *)a.v;
     p.la = a.log_alpha;
     p.w = (const __nv_bfloat16 *)a.w;
     p.init_state = a.init_state;
@@ -1379,6 +1536,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.final_state = a.final_state;
     p.T = a.T;
     p.H = a.H;
+    p.tokens = tokens;
     p.units = units;
     p.nseg = a.nseg;
     p.seg_len = a.seg_len;
@@ -1388,7 +1546,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     p.seg_s0 = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_state_offset(a.B, a.T, a.H)) : nullptr;
     p.seg_phi = a.nseg > 1 ? reinterpret_cast<float *>(ws + seg_phi_offset(a.B, a.T, a.H, a.nseg)) : nullptr;
     auto kernel = a.pre ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = ensure_dynamic_smem((const void *)kernel, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * kPairs * clusters), 1, 1);

@@ -5,11 +5,46 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <tuple>
+#include <vector>
+
 namespace gdr2 {
 
 // Chunk length of the chunkwise form ("Chunkwise training and gate-aware
 // backward", ainews.random.gg article: C = 64).
 constexpr int kChunk = 64;
+
+// Raises a kernel's dynamic shared-memory limit on the current device the
+// first time a launch there needs it, instead of on every launch (the setting
+// lasts as long as the device's context). Host only.
+inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)
+{
+    static std::mutex mu;
+    static std::vector<std::tuple<const void *, int, int>> done;  // kernel, device, bytes
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto &t : done)
+        if (std::get<0>(t) == kernel && std::get<1>(t) == dev && std::get<2>(t) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.emplace_back(kernel, dev, bytes);
+    return e;
+}
+
+// Token range [begin, end) of packed sequence n, with the offsets clamped to
+// [0, tokens] and end >= begin, so that malformed offsets cannot move a
+// kernel's reads or writes outside the token tensors.
+__device__ __forceinline__ void packed_bounds(const int32_t *cu_seqlens, int64_t n, int64_t tokens,
+                                              int64_t &begin, int64_t &end)
+{
+    int64_t s = cu_seqlens[n], e = cu_seqlens[n + 1];
+    s = s < 0 ? 0 : (s > tokens ? tokens : s);
+    e = e < s ? s : (e > tokens ? tokens : e);
+    begin = s;
+    end = e;
+}
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);

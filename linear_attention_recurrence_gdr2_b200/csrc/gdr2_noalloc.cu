@@ -21,23 +21,25 @@ constexpr size_t kNoAllocScratchBytes = (size_t)kNoAllocMaxSeqs * 4;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mutex;
+void *g_scratch_ptr[kMaxDevices];  // null until a lookup on that device succeeded
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the name itself is only a host-side stand-in).
+// Device address of g_noalloc_scratch on the current device (the name itself
+// is only a host-side stand-in). A successful lookup is kept for the life of
+// the process, which assumes the device's primary context and no
+// cudaDeviceReset in between; a failed one is not kept, so a later call
+// tries again.
 gdr2_status scratch_for_current_device(void **ptr)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDR2_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDR2_ERR_UNSUPPORTED;
-    std::call_once(g_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDR2_ERR_CUDA;
         g_scratch_ptr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return GDR2_ERR_CUDA;
+    }
     *ptr = g_scratch_ptr[dev];
     return GDR2_OK;
 }

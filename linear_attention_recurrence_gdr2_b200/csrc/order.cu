@@ -9,6 +9,7 @@
 // from cu_seqlens so the host never reads it. One CTA bitonic-sorts packed
 // (chunk count, index) keys in shared memory; above kMaxSortSeqs sequences it
 // writes the identity order instead.
+#include "common.cuh"
 #include "kernels.h"
 
 namespace gdr2 {
@@ -73,8 +74,7 @@ cudaError_t launch_order_by_length(const int32_t *cu_seqlens, int64_t num_seqs, 
     while (P < num_seqs && P <= kMaxSortSeqs) P <<= 1;
     const size_t smem = num_seqs > kMaxSortSeqs ? 0 : (size_t)P * sizeof(uint32_t);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(order_by_length_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_dynamic_smem((const void *)order_by_length_kernel, (int)smem);
         if (e != cudaSuccess) return e;
     }
     order_by_length_kernel<<<1, kSortThreads, smem, stream>>>(cu_seqlens, (int)num_seqs, order);

@@ -247,14 +247,13 @@ cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream)
     float *phi = reinterpret_cast<float *>(ws + seg_phi_offset(a.B, a.T, a.H, a.nseg));
     const __nv_bfloat16 *psi = reinterpret_cast<const __nv_bfloat16 *>(ws + seg_psi_offset());
     const int comb_smem = (int)(kStateElems * 4);
-    cudaError_t e = cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         comb_smem);
+    cudaError_t e = ensure_dynamic_smem((const void *)seg_combine_kernel, comb_smem);
     if (e != cudaSuccess) return e;
     seg_combine_kernel<<<(unsigned)(a.B * a.H), 512, comb_smem, stream>>>(s0, phi, a.final_state, a.nseg, a.H);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int fix_smem = (2 * kD + kFixTok) * kPitch;
-    e = cudaFuncSetAttribute(seg_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fix_smem);
+    e = ensure_dynamic_smem((const void *)seg_correct_kernel, fix_smem);
     if (e != cudaSuccess) return e;
     const int64_t per_seg = (a.seg_len + kFixTok * kFixTiles - 1) / (kFixTok * kFixTiles);
     const int64_t ntiles = per_seg * (a.nseg - 1);  // segments 1..nseg-1

@@ -39,6 +39,39 @@ def check_full(inp, device, label):
     assert_close(f"{label} state", sf, sf_r, inp.dtype)
 
 
+def check_full_by_head(inp, device, label):
+    """Every element of o and of the final states, the oracle run one head at
+    a time (bounded host memory); the relative L2 errors are those of the
+    whole tensors, accumulated over the heads."""
+    import torch
+    t = upload(inp, device)
+    o_d, sf_d = gdr2().chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"],
+                                 t["init_state"], t["cu_seqlens"])
+    torch.cuda.synchronize()
+    gdr2().check_device_error()
+    del t
+    H = inp.q.shape[2]
+    err = {"o": [0.0, 0.0], "state": [0.0, 0.0]}
+    worst = {"o": 0.0, "state": 0.0}
+    for h in range(H):
+        sl = lambda x: np.ascontiguousarray(x[:, :, h:h + 1])
+        s0 = np.ascontiguousarray(inp.init_state[:, h:h + 1]) if inp.init_state is not None else None
+        o_r, sf_r = oracle.forward(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha), sl(inp.b),
+                                   sl(inp.w), s0, inp.cu_seqlens)
+        o_h = o_d[:, :, h:h + 1].float().cpu().numpy()
+        sf_h = sf_d[:, h:h + 1].cpu().numpy()
+        for key, x, r in (("o", o_h, o_r), ("state", sf_h, sf_r)):
+            d = np.asarray(x, np.float64) - r
+            err[key][0] += float(np.sum(d * d))
+            err[key][1] += float(np.sum(r * r))
+            worst[key] = max(worst[key], float(np.max(np.abs(d))) if d.size else 0.0)
+            assert np.all(np.isfinite(x)), f"{label} {key}: non-finite values"
+    for key in ("o", "state"):
+        e = float(np.sqrt(err[key][0] / err[key][1]))
+        print(f"{label} {key}: rel_l2={e:.3e} max_abs={worst[key]:.3e} (tol {TOL[inp.dtype]:.0e})")
+        assert e <= TOL[inp.dtype], f"{label} {key}: rel_l2 {e:.3e} > {TOL[inp.dtype]:.0e}"
+
+
 def check_units(inp, device, units, label):
     o, sf = run_chunk(inp, device)
     for n, h in units:
@@ -167,25 +200,71 @@ def test_chunk_segment_split_matches_serial_scan(cuda_device):
 
 @pytest.mark.slow
 def test_layer_prefill_full_size(cuda_device):
-    """B=4, H=16, T=2048, d=128, bf16: six (sequence, head) units recomputed."""
-    inp = gen.layer_prefill()
-    check_units(inp, cuda_device, [(0, 0), (1, 5), (2, 9), (3, 15), (0, 13), (3, 2)], "prefill")
+    """B=4, H=16, T=2048, d=128, bf16: all 64 (sequence, head) units, every element."""
+    check_full_by_head(gen.layer_prefill(), cuda_device, "prefill")
 
 
 @pytest.mark.slow
 def test_long_context_full_size(cuda_device):
-    """B=1, H=16, T=32768, d=128, bf16, slow forgetting, nonzero initial state."""
-    inp = gen.long_context()
-    check_units(inp, cuda_device, [(0, 0), (0, 11)], "long")
+    """B=1, H=16, T=32768, d=128, bf16, slow forgetting, nonzero initial state
+    (segment-parallel scan, 2 segments): all 16 heads, every element."""
+    check_full_by_head(gen.long_context(), cuda_device, "long")
 
 
 @pytest.mark.slow
 def test_varlen_packed_full_size(cuda_device):
-    """64 packed sequences, lengths in [128, 8192], H=16, bf16, per-sequence states."""
-    inp = gen.varlen_packed()
-    lengths = np.diff(inp.cu_seqlens)
-    picks = [int(np.argmax(lengths)), int(np.argmin(lengths)), 17, 40]
-    check_units(inp, cuda_device, [(n, (3 * n) % 16) for n in picks], "varlen")
+    """64 packed sequences, lengths in [128, 8192], H=16, bf16, per-sequence
+    states: every sequence and head, every element."""
+    check_full_by_head(gen.varlen_packed(), cuda_device, "varlen")
+
+
+@pytest.mark.slow
+def test_long_single_head_sixteen_segments(cuda_device):
+    """B=1, H=1, T=32768, d=128, bf16, slow forgetting: the segment split at
+    its most segments (16 of 2048 tokens), the longest combine chain."""
+    import linear_attention_recurrence_gdr2_b200 as m
+    ws = m.workspace_size(1, 32768, 1, 128, 128, 1, m.GDR2_BF16)
+    assert ws >= 32768 * 256 + 2 * 16 * 65536  # psi and two arrays of 16 segment states
+    check_full(gen.long_context(T=32768, H=1), cuda_device, "long H=1 P=16")
+
+
+# ------------------------------------------------------- method edge cases
+def edge_case_inputs(case, dtype, d, seed):
+    """The method's degenerate settings on otherwise usual inputs (two
+    sequences of 200 tokens, three heads, nonzero initial states):
+      no_erase     b = 0: decayed linear attention (nothing is erased)
+      exact_recall b = w = 1, alpha = 1, unit keys: the delta rule at full
+                   strength, where (I + A) is least well conditioned
+      no_write     w = 0: pure erase (the state only decays and is erased)
+    """
+    inp = gen.make_inputs(2, 200, 3, d, d, dtype, seed=seed, init_std=0.05)
+    if case == "no_erase":
+        inp.b[...] = 0.0
+    elif case == "exact_recall":
+        inp.b[...] = 1.0
+        inp.w[...] = 1.0
+        inp.log_alpha[...] = 0.0
+    elif case == "no_write":
+        inp.w[...] = 0.0
+    else:
+        raise ValueError(case)
+    return inp
+
+
+@pytest.mark.parametrize("case", ["no_erase", "exact_recall", "no_write"])
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("fp32", 64), ("fp32", 128)])
+def test_method_edge_cases(cuda_device, case, dtype, d):
+    check_full(edge_case_inputs(case, dtype, d, seed=51), cuda_device, f"{case} {dtype} d={d}")
+
+
+def test_exact_recall_reads_back_the_value(cuda_device):
+    """With b = w = 1, alpha = 1 and the query equal to the key, the readout
+    is the token's own value (S_t^T k_t = v_t for a unit key): checked on the
+    GPU output itself, for fp32 inputs whose keys are unit vectors."""
+    inp = edge_case_inputs("exact_recall", "fp32", 64, seed=52)
+    inp.q[...] = inp.k
+    o, _ = run_chunk(inp, cuda_device)
+    assert rel_l2(o, inp.v.astype(np.float64)) < 1e-4
 
 
 # ------------------------------------------------------------------- decode

@@ -27,6 +27,13 @@ def test_chunk_bwd_refuses_host_tensors():
         gdr2.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["v"])
 
 
+def test_chunk_fwd_noalloc_refuses_host_tensors():
+    x = host_inputs()
+    with pytest.raises(ValueError, match="CUDA"):
+        gdr2.chunk_fwd_noalloc(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"],
+                               o=torch.zeros_like(x["v"]))
+
+
 def test_recurrent_step_refuses_host_tensors():
     z = lambda *s: torch.zeros(*s, dtype=torch.float32)
     q = z(2, 1, 64)

@@ -52,6 +52,9 @@
  *     token recurrence instead -- for the bf16 d = 128 kernel the whole
  *     (sequence, head) unit, otherwise that chunk -- which is slower but
  *     exact to fp32 rounding. Nothing is reported and nothing is clamped.
+ *     log_alpha > 0 (alpha > 1) is outside the operator's domain: the range
+ *     test reads the chunk's half sums, which bound every factor only when the
+ *     decay is monotone, so such inputs give unspecified results.
  */
 #ifndef GDR2_H_
 #define GDR2_H_

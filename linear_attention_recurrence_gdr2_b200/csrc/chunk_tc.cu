@@ -307,12 +307,13 @@ __device__ __forceinline__ UnitJob unit_job(const TcParams &prm, uint32_t cta, u
 {
     UnitJob u{false, false, 0, 0, 0, nullptr, nullptr};
     const int64_t H = prm.H;
-    const int64_t unit = (int64_t)(cta / (2 * kPairs)) * kPairs + (rank % kPairs);
-    if (unit >= prm.units) return u;
+    // (32-bit index arithmetic: the launch keeps units below 2^30 and H below 2^16)
+    const uint32_t unit = (cta / (2 * kPairs)) * kPairs + (rank % kPairs);
+    if ((int64_t)unit >= prm.units) return u;
     u.valid = true;
-    const int jobs = 2 * prm.nseg - 1;
-    const int64_t nj = unit / H;
-    u.h = unit % H;
+    const uint32_t jobs = 2 * (uint32_t)prm.nseg - 1, H32 = (uint32_t)H;
+    const uint32_t nj = unit / H32;
+    u.h = unit % H32;
     const int job = (int)(nj % jobs);
     const int64_t n = prm.order ? (int64_t)prm.order[nj / jobs] : (int64_t)(nj / jobs);
     if (prm.cu_seqlens) {
@@ -351,6 +352,7 @@ __device__ __forceinline__ UnitJob unit_job(const TcParams &prm, uint32_t cta, u
 // channels 16 (t >> 6) .. +15 of column j0 + (t & 63) in registers (the code
 // runs after the role split, where the first warpgroup keeps 40 registers).
 constexpr int kSerTok = 16;  // tokens staged in shared memory per batch
+template <bool kPre>
 __device__ __forceinline__ void serial_unit(const TcParams &prm, const UnitJob &u, int j0,
                                            unsigned char *smem, int t)
 {
@@ -389,7 +391,7 @@ __device__ __forceinline__ void serial_unit(const TcParams &prm, const UnitJob &
                 bf[0] = x.x; bf[1] = x.y; bf[2] = y.x; bf[3] = y.y;
                 lf[0] = l4.x; lf[1] = l4.y; lf[2] = l4.z; lf[3] = l4.w;
             }
-            if (prm.pre & GDR2_PROLOGUE_QK_L2NORM) {  // a warp holds one token's row
+            if (kPre && (prm.pre & GDR2_PROLOGUE_QK_L2NORM)) {  // a warp holds one token's row
                 float sq = 0.f, sk = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -410,14 +412,16 @@ __device__ __forceinline__ void serial_unit(const TcParams &prm, const UnitJob &
                 }
             }
             if (r < nb) {
-                const bool sig = (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID) != 0;
-                const bool spl = (prm.pre & GDR2_PROLOGUE_DECAY_SOFTPLUS) != 0;
+                const bool sig = kPre && (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID) != 0;
+                const bool spl = kPre && (prm.pre & GDR2_PROLOGUE_DECAY_SOFTPLUS) != 0;
                 float *vr = vec + r * 4 * kD + cb;
                 float4 al, ev;
-                al.x = expf(spl ? pre_neg_softplus(lf[0]) : lf[0]);
-                al.y = expf(spl ? pre_neg_softplus(lf[1]) : lf[1]);
-                al.z = expf(spl ? pre_neg_softplus(lf[2]) : lf[2]);
-                al.w = expf(spl ? pre_neg_softplus(lf[3]) : lf[3]);
+                // (alpha by the hardware exponential: relative error a few 1e-6 at
+                // |log alpha| = 20, far inside the fp32 bound)
+                al.x = __expf(spl ? pre_neg_softplus(lf[0]) : lf[0]);
+                al.y = __expf(spl ? pre_neg_softplus(lf[1]) : lf[1]);
+                al.z = __expf(spl ? pre_neg_softplus(lf[2]) : lf[2]);
+                al.w = __expf(spl ? pre_neg_softplus(lf[3]) : lf[3]);
                 ev.x = (sig ? pre_sigmoid(bf[0]) : bf[0]) * kf[0];
                 ev.y = (sig ? pre_sigmoid(bf[1]) : bf[1]) * kf[1];
                 ev.z = (sig ? pre_sigmoid(bf[2]) : bf[2]) * kf[2];
@@ -629,6 +633,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 // the W columns once chunk c-1's -W has been read out
                 if (c >= 1 && !wait_bar(&bars[M_UCONV], (c - 1) & 1, abort_flag, peer_abort, 15)) break;
                 if (c >= 1 && !wait_bar(&bars[M_WFREE], (c - 1) & 1, abort_flag, peer_abort, 16)) break;
+                // (T arrived by the helper's generic-proxy stores; the MMAs read it through
+                // the async proxy)
+                fence_proxy_async_smem();
                 tc_fence_after();
                 // -W rows r (M = 64, A negated): key channels of block kb -> lanes 16 kb .. 16 kb + 15
 #pragma unroll
@@ -817,13 +824,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int j = 32 * ew + lane;                       // value channel = TMEM lane
         const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
         float *vecF = reinterpret_cast<float *>(smem + kM_VECF);
+        // Range of the chunk form on key channel j, checked on the half sums that
+        // also give the state's chunk-to-chunk factor (log alpha <= 0, so g falls
+        // monotonically and T0 = g_31, T1 = g_63 - g_31 bound every |g_r - g_31|):
+        // each half within kFactorRange, and T1(c) + T0(c+1), the exponent of
+        // that factor, within kWindowRange. Past either, the pair recomputes the
+        // whole unit exactly, token by token, after this pass (serial_unit).
+        const uint32_t peer_range_flag = mapa_shared(sbase + kMISC + kRangeFlagOff, peer);
+        auto out_of_range = [&]() {
+            *range_flag = 1;
+            st_cluster_u32(peer_range_flag, 1u);
+        };
         const uint32_t zeros[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         bool ok = true;
         // master = Diag(e^{g_31 of chunk 0}) S0  (transposed: row j over key channels); O = 0
         ok = group_and(kBarEpi, 128, wait_bar(&bars[M_F0], 0, abort_flag, peer_abort, 9));
         if (ok) {
-            vecF[j] = expf(reinterpret_cast<const float *>(smem + mVEC(0))[j]);
+            const float t00 = reinterpret_cast<const float *>(smem + mVEC(0))[j];
+            vecF[j] = expf(t00);
+            if (t00 < -kFactorRange) out_of_range();
             named_bar_sync(kBarEpi, 128);
 #pragma unroll
             for (int g4 = 0; g4 < 4; ++g4) {
@@ -866,7 +886,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (!group_and(kBarEpi, 128,
                            last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag, peer_abort, 26)))
                 break;
-            vecF[j] = expf(t1c + (last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j]));
+            const float t0n = last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j];
+            vecF[j] = expf(t1c + t0n);
+            if (t1c < -kFactorRange || t0n < -kFactorRange || t1c + t0n < -kWindowRange) out_of_range();
             // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_UDONE], c & 1, abort_flag, peer_abort, 10))) break;
             tc_fence_after();
@@ -1069,7 +1091,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const float *la_s = reinterpret_cast<const float *>(smem + kH_LA);  // staged log_alpha [64][128]
         float *vecBS = reinterpret_cast<float *>(smem + kH_BSUM);          // [8][128]
         const uint32_t m_p = mapa_shared(smem_u32(&bars[M_P0]), peer);
-        const uint32_t peer_range_flag = mapa_shared(sbase + kMISC + kRangeFlagOff, peer);
         int la_issued = 0;  // log_alpha tiles staged so far (thread tp == 0)
         if (tp == 0) {
             ++la_issued;
@@ -1127,17 +1148,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
                 if (pw == 0 || pw == 4)
                     *reinterpret_cast<float4 *>(smem + hVEC(s) + (pw == 0 ? 0 : 512) + 16 * g) = half;
-                // the state passes from chunk c-1's frame to chunk c's with the one factor
-                // e^{T1(c-1) + T0(c)} (second half of the last chunk, first half of this
-                // one), which has to stay a normal fp32 number
-                if (pw == 0 && c >= 1) {
-                    const float4 t1p = *reinterpret_cast<const float4 *>(smem + hVEC(s ^ 1) + 512 + 16 * g);
-                    const float a = fminf(fminf(t1p.x + half.x, t1p.y + half.y), fminf(t1p.z + half.z, t1p.w + half.w));
-                    if (a < -kWindowRange && !*range_flag) {
-                        *range_flag = 1;
-                        st_cluster_u32(peer_range_flag, 1u);
-                    }
-                }
                 if (pw < 4) {
 #pragma unroll
                     for (int i = 7; i >= 0; --i) {
@@ -1151,19 +1161,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         run.x += la[i].x; run.y += la[i].y; run.z += la[i].z; run.w += la[i].w;
                         la[i] = make_float4(run.x * kLog2e, run.y * kLog2e, run.z * kLog2e, run.w * kLog2e);
                     }
-                }
-            }
-            // range of the factors e^{+-d}: past it (decay of more than kFactorRange
-            // within half a chunk) the whole unit is recomputed exactly, token by
-            // token, once this pass is done (see serial_unit)
-            {
-                float m = 0.f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    m = fmaxf(m, fmaxf(fmaxf(fabsf(la[i].x), fabsf(la[i].y)), fmaxf(fabsf(la[i].z), fabsf(la[i].w))));
-                if (m > kFactorRange * kLog2e && !*range_flag) {
-                    *range_flag = 1;
-                    st_cluster_u32(peer_range_flag, 1u);
                 }
             }
             // prologue: 1 / ||q_r||, 1 / ||k_r|| (a warp holds whole rows: lanes
@@ -1406,7 +1403,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                            c < 2 || wait_bar(&bars[H_TFREE0 + s], ((c >> 1) - 1) & 1, abort_flag,
                                                    peer_abort, 10)))
                 break;
-            {   // T (lower triangle incl. diagonal) -> bf16 MMA operand
+            {   // T (lower triangle incl. diagonal) -> bf16 MMA operand, stored straight into
+                // the main CTA's T buffer; the 8 KB complete on its barrier
+                const uint32_t bar = m_t + 8 * s;
+                if (tp == 0) mbar_remote_arrive_expect_tx(bar, 8192);
+                const uint32_t dst = mapa_shared(sbase + mT(s), peer);
                 const int r = tp >> 1, half = tp & 1;
                 const float *trow = sT + r * kLD + 32 * half;
 #pragma unroll
@@ -1418,16 +1419,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                         ue[e] = pack_bf16x2(s0 <= r ? trow[8 * q + 2 * e] : 0.f,
                                             s0 + 1 <= r ? trow[8 * q + 2 * e + 1] : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(smem + hT(s) + sw128_offset(r, 64 * half + 16 * q)) =
-                        make_uint4(ue[0], ue[1], ue[2], ue[3]);
+                    st_async_v4(dst + sw128_offset(r, 64 * half + 16 * q), make_uint4(ue[0], ue[1], ue[2], ue[3]), bar);
                 }
             }
-            fence_proxy_async_smem();
-            named_bar_sync(kBarPrepB, 128);
             if (tp == 0) {
-                const uint32_t bar = m_t + 8 * s;
-                mbar_remote_arrive_expect_tx(bar, 8192);
-                bulk_copy_to_cluster(mapa_shared(sbase + mT(s), peer), sbase + hT(s), 8192, bar);
                 copy_count[4 + s] += 1;
             }
         }
@@ -1460,7 +1455,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         uint32_t cta;
         asm volatile("mov.u32 %0, %%ctaid.x;" : "=r"(cta));
         const uint32_t rk = cluster_ctarank();
-        serial_unit(prm, unit_job(prm, cta, rk), rk < (uint32_t)kPairs ? 0 : 64, smem, (int)threadIdx.x);
+        serial_unit<kPre>(prm, unit_job(prm, cta, rk), rk < (uint32_t)kPairs ? 0 : 64, smem, (int)threadIdx.x);
     }
 }
 

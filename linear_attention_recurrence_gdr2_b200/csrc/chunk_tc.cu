@@ -169,13 +169,22 @@ struct TcParams {
 // Bounded wait on a barrier of this CTA (CTA-scope acquire: the peer's
 // arrives only signal, and its data arrives by bulk copies that complete on
 // this CTA's barriers). A wait that fails also raises the peer CTA's abort
-// flag, so that the whole cluster winds down.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         uint32_t peer_abort, int site) {
+// flag, so that the whole cluster winds down. Only the first (blocking)
+// probe is inlined at each wait site; the bounded loop behind it is one
+// shared function, which keeps the role loops short in instruction memory
+// (their per-chunk code is fetched again every chunk) and leaves their
+// registers to the hot path.
+__device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t peer_abort, int site) {
     WaitGuard g{kWaitNs, abort_flag, &g_chunk_tc_error};
     const bool ok = mbar_wait(bar, parity, g, site);
     if (!ok) st_cluster_u32(peer_abort, 1u);
     return ok;
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         uint32_t peer_abort, int site) {
+    if (mbar_try(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, abort_flag, peer_abort, site);
 }
 
 // Descriptor of the operand `bytes` further on in the same tile (the start
@@ -870,6 +879,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_arrive(&bars[M_SREADY_HI]);
             }
         }
+        bool chain_done = false;  // the last chunk's hand-off has completed
         for (int c = 0; ok && c < nc; ++c) {
             const int s = c & 1;
             const int64_t t0 = t_begin + 64 * c;
@@ -880,15 +890,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             float t1c = reinterpret_cast<const float *>(smem + mVEC(s))[128 + j];
             asm volatile("mov.b32 %0, %0;" : "+f"(t1c));
             const bool last = (c + 1 == nc);
-            // state scale for this chunk's hand-off, e^{g_C - g_31} and, unless last,
-            // e^{g'_31} of the next chunk (whose factors arrived long ago); the last
-            // readers of vecF finished before the previous chunk's final group barrier
-            if (!group_and(kBarEpi, 128,
-                           last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag, peer_abort, 26)))
-                break;
-            const float t0n = last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j];
-            vecF[j] = expf(t1c + t0n);
-            if (t1c < -kFactorRange || t0n < -kFactorRange || t1c + t0n < -kWindowRange) out_of_range();
             // U^T (fp32) -> bf16 pairs in TMEM for the update MMAs
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_UDONE], c & 1, abort_flag, peer_abort, 10))) break;
             tc_fence_after();
@@ -912,6 +913,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             if (te == 0) {
                 mbar_arrive(&bars[M_UCONV]);
             }
+            // state scale for this chunk's hand-off, e^{g_C - g_31} and, unless last,
+            // e^{g'_31} of the next chunk (its slot is not refilled before this
+            // chunk's state has been handed off); the last readers of vecF finished
+            // before the previous chunk's final group barrier, and the group
+            // barrier of the SDONE wait below publishes the new factors
+            if (!group_and(kBarEpi, 128,
+                           last || wait_bar(&bars[M_F0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag, peer_abort, 26)))
+                break;
+            const float t0n = last ? 0.f : reinterpret_cast<const float *>(smem + mVEC(s ^ 1))[j];
+            vecF[j] = expf(t1c + t0n);
+            if (t1c < -kFactorRange || t0n < -kFactorRange || t1c + t0n < -kWindowRange) out_of_range();
 
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_SDONE], c & 1, abort_flag, peer_abort, 11))) break;
             tc_fence_after();
@@ -967,17 +979,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                     tc_fence_before();
                     named_bar_sync(kBarEpi, 128);
                     if (te == 0) mbar_arrive(&bars[hh ? M_SREADY_HI : M_SREADY_LO]);
-                    // the fp32 master: first read again by the next chunk's update MMAs,
-                    // which wait for the U hand-off (its tc_wait_st covers these stores)
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
-                    tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
-                } else if (final_ptr) {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        final_ptr[(int64_t)(64 * hh + q) * kD + j] = __uint_as_float(m0[q]);
-                        final_ptr[(int64_t)(64 * hh + 32 + q) * kD + j] = __uint_as_float(m1[q]);
-                    }
+                    // (the master below is first read again by the next chunk's update
+                    // MMAs, which wait for the U hand-off, whose tc_wait_st covers it)
                 }
+                // the fp32 master: after the last chunk it is the final state, which
+                // is written out after the loop (off the per-chunk code)
+                tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
+                tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
             }
             // o rows of this chunk into the staging tile, from which the -W group
             // stores them to global memory; adjacent lanes (channels j, j+1) trade
@@ -1000,8 +1008,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             }
             named_bar_sync(kBarEpi, 128);
             if (te == 0) mbar_arrive(&bars[M_OFULL]);
+            if (last) chain_done = true;
         }
         tc_wait_st();  // (a master write-back may still be in flight after an abort)
+        if (chain_done && final_ptr) {
+            // final state, key channel ch (row) x value channel j: 32 key channels
+            // per TMEM load, each store coalesced over the warp's value channels
+#pragma unroll 1
+            for (int g4 = 0; g4 < 4; ++g4) {
+                uint32_t m[32];
+                tmem_ld32(tb + kTmMaster + lane_off + 32 * g4, m);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) final_ptr[(int64_t)(32 * g4 + q) * kD + j] = __uint_as_float(m[q]);
+            }
+        }
     }
     } else {
     // =========================================================================

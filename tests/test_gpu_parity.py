@@ -331,3 +331,32 @@ def test_decode_matches_chunk_forward(cuda_device):
     torch.cuda.synchronize()
     assert rel_l2(np.stack(o_d, axis=1), o_c) < 1e-4
     assert rel_l2(to_np(state), s_c) < 1e-4
+
+
+# ------------------------------------------------ malformed packed offsets
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp32", 64)])
+def test_malformed_offsets_stay_in_bounds(cuda_device, dtype, d):
+    """Packed-batch offsets that are negative, past the end or decreasing are
+    clamped to [0, tokens] by the kernels (end >= start): every write stays
+    inside o and the final states (guard rows around both are untouched) and
+    no device error is raised. The values of overlapping ranges are not
+    checked (two units then write the same rows)."""
+    import torch
+    T = 130
+    inp = gen.make_inputs(1, T, 2, d, d, dtype, seed=61, init_std=0.05)
+    t = upload(inp, cuda_device)
+    cu = torch.tensor([0, 5, 3, 500, -7, T], dtype=torch.int32, device=cuda_device)
+    N = cu.shape[0] - 1
+    g = 8
+    tdt = t["q"].dtype
+    o_big = torch.full((1, T + 2 * g, 2, d), 7.0, dtype=tdt, device=cuda_device)
+    s_big = torch.full((N + 2, 2, d, d), 7.0, dtype=torch.float32, device=cuda_device)
+    o = o_big[:, g:g + T]
+    s = s_big[1:N + 1]
+    s0 = torch.zeros((N, 2, d, d), dtype=torch.float32, device=cuda_device)
+    gdr2().chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], s0, cu, o=o, final_state=s)
+    torch.cuda.synchronize()
+    gdr2().check_device_error()
+    assert bool((o_big[:, :g] == 7.0).all()) and bool((o_big[:, g + T:] == 7.0).all())
+    assert bool((s_big[0] == 7.0).all()) and bool((s_big[N + 1] == 7.0).all())
+    assert bool(torch.isfinite(o.float()).all()) and bool(torch.isfinite(s).all())

@@ -29,7 +29,8 @@
 //     Z = w . v; -W = -(T Em) (two M=64 halves); U0^T = Z^T T^T;
 //     [U^T | O^T]  += Sm^T [-W; Qm]^T   M=128 N=128 K=128, A in TMEM
 //     [O^T | M^T]  += U^T [P^T | Km]    M=128 N=192 K=64,  A in TMEM
-//     and the epilogue (U^T to bf16, o staging, state scaling, final state).
+//     the epilogue (U^T to bf16, state scaling, final state), and O^T out of
+//     TMEM into o (16-byte stores through a staging tile).
 // Everything is computed transposed so that the value dimension (128) sits
 // on the MMA's M axis and on the 128 TMEM lanes. The fp32 state lives in the
 // main CTA's TMEM (as M = Diag(e^{g_31}) S plus the chunk's update); once per
@@ -43,7 +44,7 @@
 //   main:   0 v and w TMA producer, slot-free relay
 //           1 tcgen05.mma issuer: W, U0      2 TMEM allocator, copy-landed relay
 //           3 tcgen05.mma issuer: state chain
-//           4..7 Z      8..11 -W from TMEM, o stores      12..15 epilogue
+//           4..7 Z, O^T readout and o stores   8..11 -W from TMEM   12..15 epilogue
 //   helper: 0 q, k, b TMA producer           1 tcgen05.mma issuer: [A^T | P^T]
 //           2 TMEM allocator, factor sender   4..11 decay factors, P^T
 //           12..15 (I + A)^{-1}
@@ -117,7 +118,7 @@ constexpr uint32_t kFBytes = 32768 + 16384 + 1024;  // Em|Qm, Km, half sums
 enum {
     M_F0 = 0, M_F1, M_P0, M_P1, M_T0, M_T1, M_VFULL0, M_VFULL1, M_VFREE0, M_VFREE1, M_ZREADY0, M_ZREADY1,
     M_WDONE, M_WFREE, M_WREADY0, M_WREADY1, M_SREADY_LO, M_SREADY_HI, M_UDONE, M_UCONV, M_SDONE,
-    M_OFULL, M_OFREE,
+    M_OZERO,
     M_WTFULL, M_WTFREE,
     M_SLOTFREE0,
     M_SLOTFREE1, M_DRAIN, M_DRAIN2, M_NUM
@@ -685,6 +686,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 const uint64_t dwq = desc_at(d_wq, mEQ(s) - mEQ(0)), dpk = desc_at(d_pk, mKB(s) - mKB(0));
                 if (!spin_bar(&bars[M_WREADY0 + s], (c >> 1) & 1, abort_flag, peer_abort, 17)) break;
                 if (!spin_bar(&bars[M_SREADY_LO], c & 1, abort_flag, peer_abort, 18)) break;
+                // (the O^T columns have been read out and cleared after chunk c-1)
+                if (c >= 1 && !spin_bar(&bars[M_OZERO], (c - 1) & 1, abort_flag, peer_abort, 29)) break;
                 tc_fence_after();
                 // [U^T | O^T] += Sm^T [-W ; Qm]^T   (N = 128: -W rows then Qm rows); the
                 // state arrives in two halves of 64 key channels (K steps 0-3, 4-7)
@@ -715,15 +718,77 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         setmaxnreg_inc152();
         // ------------- Z = w . v, in place over the v tile ---------------------
         // Lane g owns value channels 4g..4g+3 (64-channel block g / 16), warp pw
-        // rows 16pw..16pw+15; rows past the chunk end are zeroed.
+        // rows 16pw..16pw+15; rows past the chunk end are zeroed. Iteration c also
+        // takes chunk c-1's O^T out of TMEM (below), one chunk behind the Z tiles,
+        // which run far ahead of the state chain.
         const int pw = warp - 4, tp = tid - 128;
         const int g = lane, kb = g >> 4;
         const uint32_t cbyte = 8 * (g & 15);
-        for (int c = 0; c < nc; ++c) {
-            const int s = c & 1;
-            const int64_t t0 = t_begin + 64 * c;
+        const int jo = 32 * pw + lane;                        // value channel = TMEM lane
+        const uint32_t lane_o = (uint32_t)(32 * pw) << 16;
+        __nv_bfloat16 *obase = zero_v ? prm.psi : prm.o;  // (an identity run writes psi)
+        // O^T of chunk cc: rows (tokens) of value channel jo as bf16 pairs, the
+        // columns cleared for the next chunk (M_OZERO), then o through the staging
+        // tile: adjacent lanes (channels j, j+1) trade halves so that the even
+        // lane writes rows 2q and the odd lane rows 2q+1 as 4-byte (j, j+1)
+        // pairs, and every row leaves in 16-byte pieces; rows past the sequence
+        // end are not written
+        auto o_out = [&](int cc) -> bool {
+            if (!group_and(kBarZ, 128, wait_bar(&bars[M_SDONE], cc & 1, abort_flag, peer_abort, 30))) return false;
+            tc_fence_after();
+            uint32_t opk[32];
+            {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tb + kTmO + lane_o, v0);
+                tmem_ld32(tb + kTmO + lane_o + 32, v1);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    opk[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
+                    opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
+                }
+            }
+            if (cc + 1 < nc) {
+                const uint32_t zeros[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                            0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                tmem_st32(tb + kTmO + lane_o, zeros);
+                tmem_st32(tb + kTmO + lane_o + 32, zeros);
+                tc_wait_st();
+            }
+            tc_fence_before();
+            named_bar_sync(kBarZ, 128);
+            if (tp == 0) mbar_arrive(&bars[M_OZERO]);
+            {
+                const bool odd = (lane & 1) != 0;
+                unsigned char *ost = smem + kM_OST + 2 * (jo & ~1);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel jo
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
+                    const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+                    const int r = 2 * q + (odd ? 1 : 0);
+                    *reinterpret_cast<uint32_t *>(ost + r * kOPitch) = pr;
+                }
+            }
+            named_bar_sync(kBarZ, 128);
+            const int64_t t0 = t_begin + 64 * cc;
             const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-            if (zero_v) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int idx = tp + 128 * i, r = idx >> 4, piece = idx & 15;
+                if (r < L) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(smem + kM_OST + r * kOPitch + 16 * piece);
+                    *reinterpret_cast<uint4 *>(obase + ((t0 + r) * H + h) * kD + 8 * piece) = v;
+                }
+            }
+            // (the staging tile is written again only after the group barrier of
+            // the next SDONE wait)
+            return true;
+        };
+        for (int c = 0; c <= nc; ++c) {
+            const int s = c & 1;
+            if (c < nc && zero_v) {
                 // Z = 0: clear the slot once its previous U0 MMA is done (that wait
                 // also paces the hand-offs, one phase per chunk and slot)
                 if (!group_and(kBarZ, 128, c < 2 || wait_bar(&bars[M_VFREE0 + s], ((c >> 1) - 1) & 1, abort_flag,
@@ -736,37 +801,40 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 }
                 named_bar_sync(kBarZ, 128);
                 if (tp == 0) mbar_arrive(&bars[M_ZREADY0 + s]);
-                continue;
-            }
-            if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5) &&
-                                           wait_bar(&bars[M_WTFULL], c & 1, abort_flag, peer_abort, 6)))
-                break;
-            unsigned char *z_tile = smem + mZ(s) + kb * 8192;
-            const unsigned char *w_tile = smem + kM_WT + kb * 8192;
+            } else if (c < nc) {
+                const int64_t t0 = t_begin + 64 * c;
+                const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
+                if (!group_and(kBarZ, 128, wait_bar(&bars[M_VFULL0 + s], (c >> 1) & 1, abort_flag, peer_abort, 5) &&
+                                               wait_bar(&bars[M_WTFULL], c & 1, abort_flag, peer_abort, 6)))
+                    break;
+                unsigned char *z_tile = smem + mZ(s) + kb * 8192;
+                const unsigned char *w_tile = smem + kM_WT + kb * 8192;
 #pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * pw + i;
-                const uint32_t off = sw128_offset(r, cbyte);
-                const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
-                const uint2 wr = *reinterpret_cast<const uint2 *>(w_tile + off);
-                const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
-                float2 w0 = bf2_to_f2(wr.x), w1 = bf2_to_f2(wr.y);
-                if (kPre && (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID)) {
-                    w0 = make_float2(pre_sigmoid(w0.x), pre_sigmoid(w0.y));
-                    w1 = make_float2(pre_sigmoid(w1.x), pre_sigmoid(w1.y));
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * pw + i;
+                    const uint32_t off = sw128_offset(r, cbyte);
+                    const uint2 vr = *reinterpret_cast<const uint2 *>(z_tile + off);
+                    const uint2 wr = *reinterpret_cast<const uint2 *>(w_tile + off);
+                    const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y);
+                    float2 w0 = bf2_to_f2(wr.x), w1 = bf2_to_f2(wr.y);
+                    if (kPre && (prm.pre & GDR2_PROLOGUE_GATE_SIGMOID)) {
+                        w0 = make_float2(pre_sigmoid(w0.x), pre_sigmoid(w0.y));
+                        w1 = make_float2(pre_sigmoid(w1.x), pre_sigmoid(w1.y));
+                    }
+                    const bool ok = r < L;
+                    uint2 oz;
+                    oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
+                    oz.y = ok ? pack_bf16x2(v1.x * w1.x, v1.y * w1.y) : 0u;
+                    *reinterpret_cast<uint2 *>(z_tile + off) = oz;
                 }
-                const bool ok = r < L;
-                uint2 oz;
-                oz.x = ok ? pack_bf16x2(v0.x * w0.x, v0.y * w0.y) : 0u;
-                oz.y = ok ? pack_bf16x2(v1.x * w1.x, v1.y * w1.y) : 0u;
-                *reinterpret_cast<uint2 *>(z_tile + off) = oz;
+                fence_proxy_async_smem();
+                named_bar_sync(kBarZ, 128);
+                if (tp == 0) {
+                    mbar_arrive(&bars[M_ZREADY0 + s]);
+                    mbar_arrive(&bars[M_WTFREE]);
+                }
             }
-            fence_proxy_async_smem();
-            named_bar_sync(kBarZ, 128);
-            if (tp == 0) {
-                mbar_arrive(&bars[M_ZREADY0 + s]);
-                mbar_arrive(&bars[M_WTFREE]);
-            }
+            if (c >= 1 && !o_out(c - 1)) break;
         }
     } else if (warp < 12) {
         setmaxnreg_inc152();
@@ -776,28 +844,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int pw = warp - 8, tp = tid - 256;
         const int rrow = 16 * pw + (lane & 15), kb = lane >> 4;
         const uint32_t h_tfree = mapa_shared(smem_u32(&bars[H_TFREE0]), peer);
-        __nv_bfloat16 *obase = zero_v ? prm.psi : prm.o;  // (an identity run writes psi)
-        // o of chunk cc from the staging tile: 16-byte pieces, 16 per row; rows
-        // past the sequence end are not written
-        auto store_o = [&](int cc) -> bool {
-            if (!group_and(kBarW, 128, wait_bar(&bars[M_OFULL], cc & 1, abort_flag, peer_abort, 30))) return false;
-            const int64_t t0 = t_begin + 64 * cc;
-            const int L = (int)(t_end - t0 < 64 ? t_end - t0 : 64);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int idx = tp + 128 * i, r = idx >> 4, piece = idx & 15;
-                if (r < L) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(smem + kM_OST + r * kOPitch + 16 * piece);
-                    *reinterpret_cast<uint4 *>(obase + ((t0 + r) * H + h) * kD + 8 * piece) = v;
-                }
-            }
-            named_bar_sync(kBarW, 128);
-            if (tp == 0) mbar_arrive(&bars[M_OFREE]);
-            return true;
-        };
-        for (int c = 0; c <= nc; ++c) {
+        for (int c = 0; c < nc; ++c) {
             const int s = c & 1;
-            if (c < nc) {
             if (!group_and(kBarW, 128, wait_bar(&bars[M_WDONE], c & 1, abort_flag, peer_abort, 8))) break;
             // the W and U0 MMAs have read T: the helper may send chunk c + 2's T
             // (only chunks the helper still sends wait for this)
@@ -822,9 +870,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 mbar_arrive(&bars[M_WFREE]);
                 mbar_arrive(&bars[M_WREADY0 + s]);
             }
-            }  // c < nc
-            // the previous chunk's o rows, staged by the epilogue
-            if (c >= 1 && !store_o(c - 1)) break;
         }
     } else {
         setmaxnreg_inc152();
@@ -927,24 +972,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
             if (!group_and(kBarEpi, 128, wait_bar(&bars[M_SDONE], c & 1, abort_flag, peer_abort, 11))) break;
             tc_fence_after();
-            // O^T row j -> registers as bf16 pairs (rows r, r+1), then the O region
-            // is zeroed for the next chunk; o is stored after the state hand-off
-            uint32_t opk[32];
-            {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tb + kTmO + lane_off, v0);
-                tmem_ld32(tb + kTmO + lane_off + 32, v1);
-                tc_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    opk[q] = pack_bf16x2(__uint_as_float(v0[2 * q]), __uint_as_float(v0[2 * q + 1]));
-                    opk[16 + q] = pack_bf16x2(__uint_as_float(v1[2 * q]), __uint_as_float(v1[2 * q + 1]));
-                }
-            }
-            if (!last) {
-                tmem_st32(tb + kTmO + lane_off, zeros);
-                tmem_st32(tb + kTmO + lane_off + 32, zeros);
-            }
             // the state, scaled, in two halves of 64 key channels: each half is
             // handed to the chain as soon as its bf16 copy is in TMEM
 #pragma unroll 1
@@ -987,27 +1014,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
                 tmem_st32(tb + kTmMaster + lane_off + 64 * hh, m0);
                 tmem_st32(tb + kTmMaster + lane_off + 64 * hh + 32, m1);
             }
-            // o rows of this chunk into the staging tile, from which the -W group
-            // stores them to global memory; adjacent lanes (channels j, j+1) trade
-            // halves so that the even lane writes rows 2q and the odd lane rows
-            // 2q+1 as 4-byte (j, j+1) pairs
-            if (c >= 1 && !group_and(kBarEpi, 128, wait_bar(&bars[M_OFREE], (c - 1) & 1, abort_flag, peer_abort, 29)))
-                break;
-            {
-                const bool odd = (lane & 1) != 0;
-                unsigned char *ost = smem + kM_OST + 2 * (j & ~1);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const uint32_t mine = opk[q];                       // rows (2q, 2q+1) of channel j
-                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                    // even lane: (row 2q: j, j+1); odd lane: (row 2q+1: j-1, j)
-                    const uint32_t pr = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
-                    const int r = 2 * q + (odd ? 1 : 0);
-                    *reinterpret_cast<uint32_t *>(ost + r * kOPitch) = pr;
-                }
-            }
-            named_bar_sync(kBarEpi, 128);
-            if (te == 0) mbar_arrive(&bars[M_OFULL]);
             if (last) chain_done = true;
         }
         tc_wait_st();  // (a master write-back may still be in flight after an abort)

@@ -259,9 +259,10 @@ gdr2_status gdr2_recurrent_step_preact(const void *q, const void *k, const void 
 gdr2_status gdr2_check_device_error(void *stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDR2_ERR_CUDA;
-    int code = 0;
+    int code = 0, seg_code = 0;
     if (gdr2::chunk_tc_read_and_clear_error(&code) != cudaSuccess) return GDR2_ERR_CUDA;
-    return code ? GDR2_ERR_DEVICE_TIMEOUT : GDR2_OK;
+    if (gdr2::seg_read_and_clear_error(&seg_code) != cudaSuccess) return GDR2_ERR_CUDA;
+    return (code || seg_code) ? GDR2_ERR_DEVICE_TIMEOUT : GDR2_OK;
 }
 
 gdr2_status gdr2_selftest_bounded_wait(uint32_t timeout_us, void *stream)

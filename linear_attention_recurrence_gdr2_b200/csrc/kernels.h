@@ -63,6 +63,9 @@ size_t seg_phi_offset(int64_t B, int64_t T, int64_t H, int nseg);
 // After the segmented chunk forward: chain the segment states, write the
 // final states and add each later segment's entry-state contribution to o.
 cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream);
+// Reads and clears the segment correction's device error word (nonzero: a
+// bounded wait gave up; the low byte is the wait site).
+cudaError_t seg_read_and_clear_error(int *code);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 

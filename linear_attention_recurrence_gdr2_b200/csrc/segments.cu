@@ -21,6 +21,9 @@
 // affine-map scan of the state, computed in fp32.)
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
+
+#include <mutex>
 
 namespace gdr2 {
 
@@ -36,177 +39,256 @@ constexpr int kMaxSegments = 16;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Per (sequence, head): S <- S0_0, then for p = 1..nseg-1 S <- Phi_p S + S0_p,
-// storing the entry state S of segment p (transposed, as bf16 hi + lo) over
-// Phi_p once that is read; finally the final state. 512 threads; thread t owns row t/4 and the 32
-// columns 4 (t%4) + 16 m + {0..3}, m = 0..7 (a warp's reads of one S row are
-// 4 adjacent 16-byte pieces: no bank conflicts).
-__global__ void __launch_bounds__(512)
-seg_combine_kernel(const float *__restrict__ s0, float *__restrict__ phi_w, float *__restrict__ final_state,
-                   int nseg, int64_t H)
+// One step of the chain of segment entry states, S_start(1) = S0_0 and
+//     S_start(p+1) = Phi_p S_start(p) + S0_p,
+// with the rows of the result split over kCombCtas CTAs per (sequence, head).
+// Step p reads S_start(p) from state slot p-1 and writes S_start(p+1) over
+// slot p (each CTA reads its own rows of S0_p before it writes them), or, after
+// the last segment, into the final state. 256 threads; thread t owns row
+// t / 16 of the CTA's 16 and the 8 columns 8 (t % 16) + {0..7}.
+constexpr int kCombRows = 16;
+constexpr int kCombCtas = kD / kCombRows;
+__global__ void __launch_bounds__(256)
+seg_combine_kernel(float *__restrict__ s0, const float *__restrict__ phi, float *__restrict__ final_state,
+                   int nseg, int p, int64_t H)
 {
-    const float *phi = phi_w;
-    extern __shared__ float4 S4[];  // the running state, [128][128] fp32
-    float *S = reinterpret_cast<float *>(S4);
+    extern __shared__ float4 comb4[];
+    float *Ss = reinterpret_cast<float *>(comb4);    // S_start(p), [128][128]
+    float *Ph = Ss + kStateElems;                    // the CTA's rows of Phi_p, [16][128]
     const int tid = threadIdx.x;
-    const int64_t h = blockIdx.x % H, n = blockIdx.x / H;
-    auto slot = [&](int p) { return ((n * nseg + p) * H + h) * kStateElems; };
-    const int r = tid >> 2, cq = 4 * (tid & 3);
-    for (int i = tid; i < (int)(kStateElems / 4); i += 512)
-        S4[i] = reinterpret_cast<const float4 *>(s0 + slot(0))[i];
+    const int64_t h = blockIdx.y, n = blockIdx.z;
+    const int r0 = kCombRows * (int)blockIdx.x;
+    auto slot = [&](int q) { return ((n * nseg + q) * H + h) * kStateElems; };
+    const float4 *src = reinterpret_cast<const float4 *>(s0 + slot(p - 1));
+    for (int i = tid; i < (int)(kStateElems / 4); i += 256) comb4[i] = src[i];
+    const float4 *prow = reinterpret_cast<const float4 *>(phi + slot(p) + (int64_t)r0 * kD);
+    for (int i = tid; i < kCombRows * kD / 4; i += 256) comb4[kStateElems / 4 + i] = prow[i];
     __syncthreads();
-    for (int p = 1; p < nseg; ++p) {
-        float4 acc[8];
-        const float *s0p = s0 + slot(p) + r * kD + cq;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m] = *reinterpret_cast<const float4 *>(s0p + 16 * m);
-        const float *phr = phi + slot(p) + r * kD;
-#pragma unroll 4
-        for (int k = 0; k < kD; ++k) {
-            const float a = phr[k];
-            const float *srow = S + k * kD + cq;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float4 x = *reinterpret_cast<const float4 *>(srow + 16 * m);
-                acc[m].x = fmaf(a, x.x, acc[m].x);
-                acc[m].y = fmaf(a, x.y, acc[m].y);
-                acc[m].z = fmaf(a, x.z, acc[m].z);
-                acc[m].w = fmaf(a, x.w, acc[m].w);
-            }
-        }
-        __syncthreads();  // every read of S and of Phi_p for this step is done
-        // entry state of segment p, transposed and split into bf16 hi + lo, over
-        // Phi_p (no longer needed): [hi: 128 x 128][lo: 128 x 128], element (j, k) = S[k][j]
-        __nv_bfloat16 *sth = reinterpret_cast<__nv_bfloat16 *>(phi_w + slot(p));
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float4 x = *reinterpret_cast<const float4 *>(S + r * kD + cq + 16 * m);
-            const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = cq + 16 * m + e;
-                const __nv_bfloat16 hi = __float2bfloat16_rn(xs[e]);
-                sth[j * kD + r] = hi;
-                sth[kStateElems + j * kD + r] = __float2bfloat16_rn(xs[e] - __bfloat162float(hi));
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < 8; ++m) *reinterpret_cast<float4 *>(S + r * kD + cq + 16 * m) = acc[m];
-        __syncthreads();
+    const int rr = tid >> 4, c8 = 8 * (tid & 15);
+    const float *s0r = s0 + slot(p) + (int64_t)(r0 + rr) * kD + c8;
+    const float4 b0 = *reinterpret_cast<const float4 *>(s0r), b1 = *reinterpret_cast<const float4 *>(s0r + 4);
+    float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll 8
+    for (int k = 0; k < kD; ++k) {
+        const float a = Ph[rr * kD + k];
+        const float4 x0 = *reinterpret_cast<const float4 *>(Ss + k * kD + c8);
+        const float4 x1 = *reinterpret_cast<const float4 *>(Ss + k * kD + c8 + 4);
+        acc[0] = fmaf(a, x0.x, acc[0]); acc[1] = fmaf(a, x0.y, acc[1]);
+        acc[2] = fmaf(a, x0.z, acc[2]); acc[3] = fmaf(a, x0.w, acc[3]);
+        acc[4] = fmaf(a, x1.x, acc[4]); acc[5] = fmaf(a, x1.y, acc[5]);
+        acc[6] = fmaf(a, x1.z, acc[6]); acc[7] = fmaf(a, x1.w, acc[7]);
     }
-    if (final_state) {
-        float *dst = final_state + (n * H + h) * kStateElems + r * kD + cq;
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<float4 *>(dst + 16 * m) = *reinterpret_cast<const float4 *>(S + r * kD + cq + 16 * m);
+    float *dst = p + 1 < nseg ? s0 + slot(p) : (final_state ? final_state + (n * H + h) * kStateElems : nullptr);
+    if (dst) {
+        float *d = dst + (int64_t)(r0 + rr) * kD + c8;
+        *reinterpret_cast<float4 *>(d) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(d + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 
-constexpr int kFixTok = 64;     // tokens per tile (4 warps x 16 rows)
-constexpr int kFixTiles = 16;   // tiles per CTA (the entry state is staged once per 1024 tokens)
-constexpr int kPitch = 272;     // bytes per staged 128-element bf16 row (16 B pad: ldmatrix
-                                // rows of one 8x8 matrix fall in distinct bank groups)
+// ---- the correction o_t += S_start(p)^T psi_t on tcgen05 -------------------
+// Per 128-token tile of segment p >= 1: D (tokens x 128 out channels, fp32 in
+// TMEM) = Psi (tokens x 128 k, bf16) * S_start(p), with S_start(p) (fp32,
+// state slot p-1 after the combine steps) split into bf16 hi and lo parts and
+// staged as the MMA's B operand in its MN-major layout (rows k, output
+// channels contiguous, as S is stored); both parts accumulate into the same D
+// (the product keeps about 16 mantissa bits of S). One CTA stages S once and
+// runs up to kCorrTiles tiles of one
+// (sequence, head): warp 0 loads Psi tiles by TMA (two slots), warp 1 issues
+// the 16 MMAs of a tile into one of two TMEM accumulators, warps 4-7 add the
+// accumulator to o (thread = token row = TMEM lane). Every wait is bounded.
+constexpr int kCorrRows = 128;     // tokens per tile (the MMA's M)
+constexpr int kCorrTiles = 16;     // tiles per CTA: S^T is staged once per 2048 tokens
+constexpr int kCorrThreads = 256;
+constexpr uint32_t kCB = 0;        // S [part hi, lo][j half][128 k rows x 128 B], 64 KB
+constexpr uint32_t kCA = 65536;    // Psi slots [2][k half][128 rows x 128 B], 32 KB each
+constexpr uint32_t kCBar = 131072;
+enum { C_FULL0 = 0, C_FULL1, C_FREE0, C_FREE1, C_ACC0, C_ACC1, C_ACCFREE0, C_ACCFREE1, C_DRAIN, C_NUM };
+constexpr uint32_t kCMisc = kCBar + C_NUM * 8;      // TMEM base, abort flag
+constexpr uint32_t kCorrSmem = kCMisc + 16 + 1024;  // + alignment slack
+constexpr uint64_t kCorrWaitNs = 1000000000ull;     // one second per wait
+constexpr uint32_t kBarEpiC = 1;                    // named barrier of the epilogue warps
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+__device__ int g_seg_error;
+
+// Bounded wait: one blocking probe, then the timed loop (which records `site`
+// in the error word and raises the CTA's abort flag when the limit passes).
+__device__ __forceinline__ bool cwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int site) {
+    if (sm100::mbar_try(bar, parity)) return true;
+    sm100::WaitGuard g{kCorrWaitNs, abort_flag, &g_seg_error};
+    return sm100::mbar_wait(bar, parity, g, site);
 }
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+// Barrier over an n-thread group that ANDs one predicate across it.
+__device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
+    uint32_t r;
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
+    return r != 0;
 }
 
-// o_t += S_start(p)^T psi_t for the tokens of segments p >= 1, on the tensor
-// cores: O_tile (tokens x 128) += Psi_tile (tokens x 128, bf16) * S with
-// S = S_hi + S_lo split into two bf16 parts (so the product keeps about 16
-// mantissa bits of S) and fp32 accumulation. CTA: up to 256 tokens of one
-// (sequence, head) inside one segment; warp w: 16 tokens of each 64-token
-// tile, all 128 output channels (16 n-tiles of 8).
-__global__ void __launch_bounds__(128)
-seg_correct_kernel(__nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ psi,
-                   const float *__restrict__ sth_f, int nseg, int64_t seg_len, int64_t T, int64_t H)
+__global__ void __launch_bounds__(kCorrThreads, 1)
+seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *__restrict__ o,
+                   const float *__restrict__ sst, int nseg, int64_t seg_len, int64_t T, int64_t H)
 {
-    extern __shared__ __align__(16) unsigned char fix_smem[];
-    // (each state slot holds 64 KB: the bf16 hi and lo halves of S^T)
-    const __nv_bfloat16 *sth = reinterpret_cast<const __nv_bfloat16 *>(sth_f);
-    unsigned char *st_hi = fix_smem;                  // S^T hi: [128 out channels][128 k] bf16, kPitch
-    unsigned char *st_lo = fix_smem + kD * kPitch;    // S^T lo
-    unsigned char *pt = fix_smem + 2 * kD * kPitch;   // psi tile: [64 tokens][128 k] bf16, kPitch
+    using namespace sm100;
+    extern __shared__ __align__(1024) unsigned char corr_smem_raw[];
+    unsigned char *smem = corr_smem_raw + ((1024u - (smem_u32(corr_smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kCBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kCMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kCMisc + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t h = blockIdx.y, n = blockIdx.z;
-    const int64_t per_seg = (seg_len + kFixTok * kFixTiles - 1) / (kFixTok * kFixTiles);
+    const int64_t per_seg = (seg_len + kCorrRows * kCorrTiles - 1) / (kCorrRows * kCorrTiles);
     const int p = 1 + (int)(blockIdx.x / per_seg);
-    const int64_t tb = p * seg_len + (int64_t)(blockIdx.x % per_seg) * kFixTok * kFixTiles;  // first token
+    const int64_t tb = p * seg_len + (int64_t)(blockIdx.x % per_seg) * kCorrRows * kCorrTiles;  // first token
     const int64_t seg_end = (p + 1) * seg_len < T ? (p + 1) * seg_len : T;
-    if (tb >= seg_end) return;
-    // stage S^T hi and lo (written by the combine step, bf16 [j][k]), 16-byte pieces
-    const uint4 *src = reinterpret_cast<const uint4 *>(sth + ((n * nseg + p) * H + h) * 2 * kStateElems);
-    for (int i = tid; i < 2 * kD * kD / 8; i += 128) {
-        const int row = i >> 4, piece = i & 15;  // rows 0-127 hi, 128-255 lo
-        *reinterpret_cast<uint4 *>(fix_smem + row * kPitch + 16 * piece) = src[i];
-    }
-    // ldmatrix lane addresses: A (psi rows of this warp), B (S^T rows = output channels)
-    const int a_row = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1), a_k = 8 * (lane >> 4);
-    const int b_row = (lane & 7) + 8 * (lane >> 4), b_k = 8 * ((lane >> 3) & 1);
-    const uint32_t a_base = smem_addr(pt) + a_row * kPitch + 2 * a_k;
-    const uint32_t bh_base = smem_addr(st_hi) + b_row * kPitch + 2 * b_k;
-    const uint32_t bl_base = smem_addr(st_lo) + b_row * kPitch + 2 * b_k;
-    const int g = lane >> 2, t4 = lane & 3;
-    for (int tile = 0; tile < kFixTiles; ++tile) {
-        const int64_t t0 = tb + tile * kFixTok;
-        if (t0 >= seg_end) break;
-        __syncthreads();  // (S staged / previous tile's psi consumed)
-        for (int i = tid; i < kFixTok * kD / 8; i += 128) {  // psi rows, 16 B pieces
-            const int rr = i >> 4, piece = i & 15;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t0 + rr < seg_end)
-                v = *reinterpret_cast<const uint4 *>(psi + ((n * T + t0 + rr) * H + h) * kD + 8 * piece);
-            *reinterpret_cast<uint4 *>(pt + rr * kPitch + 16 * piece) = v;
-        }
-        __syncthreads();
-        float acc[16][4];
+    if (p >= nseg || tb >= seg_end) return;  // (the same for every thread of the CTA)
+    const int64_t left = (seg_end - tb + kCorrRows - 1) / kCorrRows;
+    const int ntiles = left < kCorrTiles ? (int)left : kCorrTiles;
+
+    // S_start(p) (fp32 [k][j]) as bf16 hi and lo into the 128B-swizzled MN-major
+    // layout: rows k, 64 output channels per 128-byte row, channel halves apart
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(sst + ((n * nseg + p - 1) * H + h) * kStateElems);
+        for (int i = tid; i < (int)(kStateElems / 4); i += kCorrThreads) {
+            const int k = i >> 5, j = 4 * (i & 31);
+            const float4 x = src[i];
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+            uint32_t hi[2], lo[2];
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
-        for (int kk = 0; kk < kD; kk += 16) {
-            uint32_t a[4];
-            ldmatrix_x4(a, a_base + 2 * kk);
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {  // n-tile pairs
-                uint32_t bh[4], bl[4];
-                ldmatrix_x4(bh, bh_base + np * 16 * kPitch + 2 * kk);
-                ldmatrix_x4(bl, bl_base + np * 16 * kPitch + 2 * kk);
-                mma_bf16_16816(acc[2 * np], a, bh[0], bh[1]);
-                mma_bf16_16816(acc[2 * np], a, bl[0], bl[1]);
-                mma_bf16_16816(acc[2 * np + 1], a, bh[2], bh[3]);
-                mma_bf16_16816(acc[2 * np + 1], a, bl[2], bl[3]);
+            for (int e = 0; e < 2; ++e) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(xs[2 * e]), h1 = __float2bfloat16_rn(xs[2 * e + 1]);
+                hi[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+                lo[e] = pack_bf16x2(xs[2 * e] - __bfloat162float(h0), xs[2 * e + 1] - __bfloat162float(h1));
             }
+            const uint32_t off = (j >> 6) * 16384 + sw128_offset(k, 2 * (j & 63));
+            *reinterpret_cast<uint2 *>(smem + kCB + off) = make_uint2(hi[0], hi[1]);
+            *reinterpret_cast<uint2 *>(smem + kCB + 32768 + off) = make_uint2(lo[0], lo[1]);
         }
-        // o (rows g, g+8 of this warp's 16; channels 8 nt + 2 t4, +1) += acc
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int64_t t = t0 + 16 * warp + g + 8 * half;
-            if (t >= seg_end) continue;
-            __nv_bfloat16 *orow = o + ((n * T + t) * H + h) * kD + 2 * t4;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                __nv_bfloat162 *po = reinterpret_cast<__nv_bfloat162 *>(orow + 8 * nt);
-                const float2 f = __bfloat1622float2(*po);
-                *po = __floats2bfloat162_rn(f.x + acc[nt][2 * half], f.y + acc[nt][2 * half + 1]);
+        fence_proxy_async_smem();  // (read next by the MMAs, through the async proxy)
+    }
+    if (tid == 0) {
+        for (int i = 0; i < C_NUM; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) prefetch_tensormap(&map_psi);
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- Psi tiles by TMA (two slots) ----
+        if (lane == 0) {
+            int issued0 = 0, issued1 = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !cwait(&bars[C_FREE0 + s], ((i >> 1) - 1) & 1, abort_flag, 40)) break;
+                const int z = (int)(n * T + tb + (int64_t)kCorrRows * i);
+                mbar_arrive_expect_tx(&bars[C_FULL0 + s], 32768);
+                for (int half = 0; half < 2; ++half)
+                    tma_load_3d(smem + kCA + s * 32768 + half * 16384, &map_psi, &bars[C_FULL0 + s], 64 * half,
+                                (int)h, z);
+                (s ? issued1 : issued0) = (i >> 1) + 1;
             }
+            // (loads still in flight after an abort land before the CTA exits)
+            if (issued0 > 0) { volatile int nf = 0; WaitGuard g{kCorrWaitNs, &nf, &g_seg_error}; mbar_wait(&bars[C_FULL0], (issued0 - 1) & 1, g, 41); }
+            if (issued1 > 0) { volatile int nf = 0; WaitGuard g{kCorrWaitNs, &nf, &g_seg_error}; mbar_wait(&bars[C_FULL1], (issued1 - 1) & 1, g, 41); }
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer: D[a] = Psi S_hi + Psi S_lo ----
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);  // A K-major, B MN-major
+            const uint64_t da = smem_desc_sw128(sbase + kCA, 16, 1024);
+            const uint64_t db = smem_desc_sw128(sbase + kCB, 16384, 1024);
+            for (int i = 0; i < ntiles; ++i) {
+                const int s = i & 1;
+                if (!cwait(&bars[C_FULL0 + s], (i >> 1) & 1, abort_flag, 42)) break;
+                if (i >= 2 && !cwait(&bars[C_ACCFREE0 + s], ((i >> 1) - 1) & 1, abort_flag, 43)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        // A: 16 k columns = 32 bytes of a row (k halves 16 KB apart);
+                        // B: 16 k rows = 2 KB
+                        const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tbase + 128 * s, da + ((s * 32768 + ka) >> 4), db + ((part * 32768 + kk * 2048) >> 4),
+                               idesc, (part | kk) != 0);
+                    }
+                tc_commit(&bars[C_FREE0 + s]);
+                tc_commit(&bars[C_ACC0 + s]);
+            }
+            tc_commit(&bars[C_DRAIN]);
+            volatile int nf = 0;
+            WaitGuard g{kCorrWaitNs, &nf, &g_seg_error};
+            mbar_wait(&bars[C_DRAIN], 0, g, 44);
+        }
+    } else if (warp >= 4) {
+        // ---- o rows += D rows (thread = token row = TMEM lane) ----
+        const int q4 = warp & 3, row = 32 * q4 + lane, te = tid - 128;
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i & 1;
+            if (!group_all(kBarEpiC, 128, cwait(&bars[C_ACC0 + s], (i >> 1) & 1, abort_flag, 45))) break;
+            tc_fence_after();
+            const int64_t t = tb + (int64_t)kCorrRows * i + row;
+            __nv_bfloat16 *orow = o + ((n * T + t) * H + h) * kD;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tbase + 128 * s + 32 * q + lane_off, v);
+                tc_wait_ld();
+                if (t < seg_end) {
+                    uint4 *po = reinterpret_cast<uint4 *>(orow + 32 * q);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint4 x = po[e];
+                        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[c]));
+                            w[c] = pack_bf16x2(f.x + __uint_as_float(v[8 * e + 2 * c]),
+                                               f.y + __uint_as_float(v[8 * e + 2 * c + 1]));
+                        }
+                        po[e] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(kBarEpiC, 128);
+            if (te == 0) mbar_arrive(&bars[C_ACCFREE0 + s]);
         }
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tbase, 256);
 }
 
 }  // namespace
+
+typedef CUresult (*EncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                             const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+cudaError_t seg_read_and_clear_error(int *code)
+{
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_seg_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_seg_error, &zero, sizeof(int));
+}
 
 size_t seg_psi_offset() { return 0; }
 
@@ -246,20 +328,44 @@ cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream)
     float *s0 = reinterpret_cast<float *>(ws + seg_state_offset(a.B, a.T, a.H));
     float *phi = reinterpret_cast<float *>(ws + seg_phi_offset(a.B, a.T, a.H, a.nseg));
     const __nv_bfloat16 *psi = reinterpret_cast<const __nv_bfloat16 *>(ws + seg_psi_offset());
-    const int comb_smem = (int)(kStateElems * 4);
+    const int comb_smem = (int)((kStateElems + kCombRows * kD) * 4);
     cudaError_t e = ensure_dynamic_smem((const void *)seg_combine_kernel, comb_smem);
     if (e != cudaSuccess) return e;
-    seg_combine_kernel<<<(unsigned)(a.B * a.H), 512, comb_smem, stream>>>(s0, phi, a.final_state, a.nseg, a.H);
-    e = cudaGetLastError();
+    for (int p = 1; p < a.nseg; ++p) {  // (each step reads the previous one's result)
+        seg_combine_kernel<<<dim3(kCombCtas, (unsigned)a.H, (unsigned)a.B), 256, comb_smem, stream>>>(
+            s0, phi, a.final_state, a.nseg, p, a.H);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // Psi [B*T tokens, H, 128] bf16 as a 3-D map; box = 128 tokens x 1 head x 64 channels
+    static std::once_flag once;
+    static EncodeFn enc = nullptr;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fp = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            enc = reinterpret_cast<EncodeFn>(fp);
+    });
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map_psi;
+    const int64_t tokens = a.B * a.T;
+    if (tokens > 0x7fffffffLL) return cudaErrorInvalidValue;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)a.H, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)(a.H * kD * 2)};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kCorrRows};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&map_psi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(psi), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    e = ensure_dynamic_smem((const void *)seg_correct_kernel, (int)kCorrSmem);
     if (e != cudaSuccess) return e;
-    const int fix_smem = (2 * kD + kFixTok) * kPitch;
-    e = ensure_dynamic_smem((const void *)seg_correct_kernel, fix_smem);
-    if (e != cudaSuccess) return e;
-    const int64_t per_seg = (a.seg_len + kFixTok * kFixTiles - 1) / (kFixTok * kFixTiles);
-    const int64_t ntiles = per_seg * (a.nseg - 1);  // segments 1..nseg-1
-    dim3 grid((unsigned)ntiles, (unsigned)a.H, (unsigned)a.B);
-    seg_correct_kernel<<<grid, 128, fix_smem, stream>>>(static_cast<__nv_bfloat16 *>(a.o), psi, phi, a.nseg,
-                                                       a.seg_len, a.T, a.H);
+    const int64_t per_seg = (a.seg_len + kCorrRows * kCorrTiles - 1) / (kCorrRows * kCorrTiles);
+    const int64_t nblk = per_seg * (a.nseg - 1);  // segments 1..nseg-1
+    dim3 grid((unsigned)nblk, (unsigned)a.H, (unsigned)a.B);
+    seg_correct_kernel<<<grid, kCorrThreads, kCorrSmem, stream>>>(map_psi, static_cast<__nv_bfloat16 *>(a.o), s0,
+                                                                 a.nseg, a.seg_len, a.T, a.H);
     return cudaGetLastError();
 }
 

@@ -14,6 +14,9 @@ Pinned by: tests/test_oracle_pins.py (KDA and Gated DeltaNet reductions,
 exact recall, b=0 closed form, brute-force transition products, the
 fast-weight argmin identity, state passing, varlen splitting, linearity; the
 prologue against scipy's logistic function, numpy's logaddexp and norm);
+tests/test_qed_oracle.py (the QED reading: its reductions to the plain rule,
+the annihilation of both erase directions, brute-force products; PARITY
+UNPINNED against the paper, which does not print the update);
 tests/test_backward_oracle.py (the backward against central finite
 differences of the forward, linearity in the cotangents, planted mistakes).
 """
@@ -64,6 +67,11 @@ def _load():
                 _D, _D, _D, _D, _D, _D, _D,
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                 _D, ctypes.c_int]
+            lib.gdr2_oracle_qed_forward.restype = ctypes.c_int
+            lib.gdr2_oracle_qed_forward.argtypes = [
+                _D, _D, _D, _D, _D, _D, _D, _D, ctypes.c_int, _D, _I64,
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                ctypes.c_int64, ctypes.c_int64, _D, _D, ctypes.c_int]
             lib.gdr2_oracle_max_threads.restype = ctypes.c_int
             lib.gdr2_oracle_max_threads.argtypes = []
             _lib = lib
@@ -116,6 +124,55 @@ def forward(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None,
         B, T, H, dk, dv, N, _p(o), _p(sf), int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle forward rejected its arguments (code {rc})")
+    return o, sf
+
+
+QED_GATE = 1      # gate the query-derived erase by b_t
+QED_PROJECT = 2   # project its direction orthogonal to k_t
+QED_FULL = QED_GATE | QED_PROJECT
+
+
+def qed_forward(q, k, v, log_alpha, b, w, strength, direction=None, flags: int = QED_FULL,
+                init_state=None, cu_seqlens=None, num_threads: int = 0):
+    """Token-by-token fp64 forward of Gated Delta Rule-2 with the QED second
+    erase direction ("The Query Knows What to Forget", thelatestinai.com
+    listing: abstract, Table 1). PARITY UNPINNED against the paper, which does
+    not print the update: this is the reading in gdr2_oracle.c's QED section
+    (a unit direction from the query, or from `direction` [H, d_k], projected
+    orthogonal to k_t with flags & QED_PROJECT, erased with strength
+    `strength` [H] and, with flags & QED_GATE, the erase gate b_t).
+
+    Shapes and return values as forward()."""
+    q, k, v, la, b, w = (_f64(x) for x in (q, k, v, log_alpha, b, w))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, x, d in (("k", k, dk), ("log_alpha", la, dk), ("b", b, dk),
+                       ("v", v, dv), ("w", w, dv)):
+        if x.shape != (B, T, H, d):
+            raise ValueError(f"{name} has shape {x.shape}, expected {(B, T, H, d)}")
+    lam = _f64(strength).reshape(-1)
+    if lam.shape != (H,):
+        raise ValueError(f"strength has shape {lam.shape}, expected ({H},)")
+    dirs = _f64(direction) if direction is not None else None
+    if dirs is not None and dirs.shape != (H, dk):
+        raise ValueError(f"direction has shape {dirs.shape}, expected {(H, dk)}")
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        cu = None
+        N = B
+    s0 = _f64(init_state) if init_state is not None else None
+    if s0 is not None and s0.shape != (N, H, dk, dv):
+        raise ValueError(f"init_state has shape {s0.shape}, expected {(N, H, dk, dv)}")
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().gdr2_oracle_qed_forward(
+        _p(q), _p(k), _p(v), _p(la), _p(b), _p(w), _p(lam), _p(dirs), int(flags), _p(s0),
+        cu.ctypes.data_as(_I64) if cu is not None else None,
+        B, T, H, dk, dv, N, _p(o), _p(sf), int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle QED forward rejected its arguments (code {rc})")
     return o, sf
 
 

@@ -178,6 +178,145 @@ int gdr2_oracle_step(const double *q, const double *k, const double *v,
     return failed ? -2 : 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * QED: a second erase direction derived from the query ("The Query Knows
+ * What to Forget: A Second Erase Direction for Linear Attention",
+ * thelatestinai.com listing: abstract and Table 1). The page names the parts
+ * of the correction (a direction from the query, projected orthogonal to the
+ * key, gated by b_t, with a per-head strength) but does not print its
+ * equation (6); this is the plain reading recorded in the design notes,
+ * PARITY UNPINNED against the paper (pinned only by the reading's own
+ * invariants and reductions):
+ *
+ *   src_t = q_t, or a fixed per-head direction r_h (the control arm)
+ *   p_t   = src_t - (k_t.src_t / k_t.k_t) k_t      (projection P^perp_{k_t};
+ *                                                   p_t = src_t if unprojected
+ *                                                   or k_t = 0)
+ *   u_t   = p_t / |p_t|   (0 when |p_t|^2 <= 1e-12 |src_t|^2)
+ *   f_t   = b_t . u_t     (u_t if ungated)
+ *   S_t   = (I - k_t (b_t . k_t)^T - lambda_h u_t f_t^T) Diag(alpha_t) S_{t-1}
+ *           + k_t (w_t . v_t)^T,           o_t = S_t^T q_t.
+ *
+ * flags: bit 0 gate the correction by b_t, bit 1 project orthogonal to k_t.
+ * ------------------------------------------------------------------------ */
+#define QED_GATE 1
+#define QED_PROJECT 2
+
+/* One QED token on one (sequence, head) state; scratch: 3*d_v + d_k doubles. */
+static void qed_token(double *S, const double *q, const double *k, const double *la,
+                      const double *b, const double *v, const double *w,
+                      const double *dir, double lambda, int flags, double *o,
+                      int64_t dk, int64_t dv, double *scratch)
+{
+    double *read_k = scratch;           /* (b.k)^T D S, length d_v */
+    double *read_u = scratch + dv;      /* f^T D S, length d_v     */
+    double *resid = scratch + 2 * dv;   /* z - read_k, length d_v  */
+    double *u = scratch + 3 * dv;       /* erase direction, d_k    */
+
+    /* D_t S_{t-1} */
+    for (int64_t c = 0; c < dk; ++c) {
+        double a = exp(la[c]);
+        double *row = S + c * dv;
+        for (int64_t j = 0; j < dv; ++j) row[j] *= a;
+    }
+    /* u_t: the source direction, projected orthogonal to k_t, normalised */
+    const double *src = dir ? dir : q;
+    double kk = 0.0, ks = 0.0, ss = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+        kk += k[c] * k[c];
+        ks += k[c] * src[c];
+        ss += src[c] * src[c];
+    }
+    double coef = ((flags & QED_PROJECT) && kk > 0.0) ? ks / kk : 0.0;
+    double pp = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+        u[c] = src[c] - coef * k[c];
+        pp += u[c] * u[c];
+    }
+    double inv = (pp > 1e-12 * ss && pp > 0.0) ? 1.0 / sqrt(pp) : 0.0;
+    for (int64_t c = 0; c < dk; ++c) u[c] *= inv;
+    /* both reads of the decayed state, before either edit */
+    for (int64_t j = 0; j < dv; ++j) read_k[j] = read_u[j] = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+        double e = b[c] * k[c];
+        double f = (flags & QED_GATE) ? b[c] * u[c] : u[c];
+        const double *row = S + c * dv;
+        for (int64_t j = 0; j < dv; ++j) {
+            read_k[j] += e * row[j];
+            read_u[j] += f * row[j];
+        }
+    }
+    /* S <- S - k read_k^T - lambda u read_u^T + k z^T */
+    for (int64_t j = 0; j < dv; ++j) resid[j] = w[j] * v[j] - read_k[j];
+    for (int64_t c = 0; c < dk; ++c) {
+        double *row = S + c * dv;
+        double lu = lambda * u[c];
+        for (int64_t j = 0; j < dv; ++j) row[j] += k[c] * resid[j] - lu * read_u[j];
+    }
+    /* o_t = S_t^T q_t */
+    for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
+    for (int64_t c = 0; c < dk; ++c) {
+        const double *row = S + c * dv;
+        for (int64_t j = 0; j < dv; ++j) o[j] += q[c] * row[j];
+    }
+}
+
+/* Whole-sequence QED forward; arguments as gdr2_oracle_forward, plus
+ * lambda [H] (per-head strength), dir [H, d_k] (fixed directions, or NULL for
+ * the query) and flags. */
+int gdr2_oracle_qed_forward(const double *q, const double *k, const double *v,
+                            const double *log_alpha, const double *b,
+                            const double *w, const double *lambda, const double *dir,
+                            int flags, const double *init_state,
+                            const int64_t *cu_seqlens, int64_t B, int64_t T,
+                            int64_t H, int64_t dk, int64_t dv, int64_t num_seqs,
+                            double *o, double *final_state, int num_threads)
+{
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || !lambda) return -1;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 0 || cu_seqlens[0] != 0 ||
+            cu_seqlens[num_seqs] != T)
+            return -1;
+        for (int64_t n = 0; n < num_seqs; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    } else if (num_seqs != B) {
+        return -1;
+    }
+    const int64_t units = num_seqs * H;
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t n = u / H, h = u % H;
+        int64_t t0 = cu_seqlens ? cu_seqlens[n] : n * T;
+        int64_t t1 = cu_seqlens ? cu_seqlens[n + 1] : n * T + T;
+        double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)(3 * dv + dk));
+        if (!S || !scratch) {
+            free(S);
+            free(scratch);
+            failed = 1;
+            continue;
+        }
+        if (init_state)
+            memcpy(S, init_state + u * dk * dv, sizeof(double) * (size_t)(dk * dv));
+        else
+            memset(S, 0, sizeof(double) * (size_t)(dk * dv));
+        for (int64_t t = t0; t < t1; ++t) {
+            const int64_t rk = (t * H + h) * dk, rv = (t * H + h) * dv;
+            qed_token(S, q + rk, k + rk, log_alpha + rk, b + rk, v + rv, w + rv,
+                      dir ? dir + h * dk : NULL, lambda[h], flags, o + rv, dk, dv, scratch);
+        }
+        if (final_state)
+            memcpy(final_state + u * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
+        free(S);
+        free(scratch);
+    }
+    return failed ? -2 : 0;
+}
+
 /* Number of threads an OpenMP parallel region would use (1 without OpenMP). */
 int gdr2_oracle_max_threads(void)
 {

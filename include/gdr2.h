@@ -311,6 +311,47 @@ gdr2_status gdr2_recurrent_step_preact(const void *q, const void *k, const void 
                                        void *stream);
 
 /*
+ * gdr2_qed_fwd -- forward with the QED second erase direction (a reading).
+ *
+ * "The Query Knows What to Forget: A Second Erase Direction for Linear
+ * Attention" (thelatestinai.com listing; abstract and Table 1) adds to the
+ * key-directed erase of Gated Delta Rule-2 a second erase direction derived
+ * from the query and orthogonal to the key, gated by b_t, with a per-head
+ * strength (its Table 4 sweeps the strength at inference). The page does not
+ * print the update (its equation (6)); this call computes the plain reading,
+ * per (sequence, head), token by token:
+ *
+ *   src = q_t, or direction[h] when `direction` is given (the paper's
+ *         fixed-direction control arm)
+ *   p   = src - (k_t.src / k_t.k_t) k_t   with GDR2_QED_PROJECT (else src)
+ *   u   = p / |p|                          (0 when |p|^2 <= 1e-12 |src|^2)
+ *   f   = b_t . u                          with GDR2_QED_GATE (else u)
+ *   S_t = (I - k_t (b_t . k_t)^T - strength[h] u f^T) Diag(exp(log_alpha_t)) S_{t-1}
+ *         + k_t (w_t . v_t)^T
+ *   o_t = S_t^T q_t
+ *
+ * Flags 0 .. 3 select the paper's Table 1 arms (GDR2_QED_GATE |
+ * GDR2_QED_PROJECT is the full variant); strength 0 is exactly the plain rule.
+ *
+ * Arguments: token tensors, init_state, cu_seqlens, B, T, H, num_seqs, dtype,
+ * o and final_state exactly as gdr2_chunk_fwd (d_k = d_v = 64 or 128;
+ * no workspace). strength: device fp32 [H]. direction: device fp32 [H, d_k]
+ * or NULL (the query). The state and all arithmetic are fp32 on the CUDA
+ * cores, one CTA per (sequence, head, 32 value columns), tokens in order: a
+ * reference-grade path, not a tuned one. Returns GDR2_ERR_INVALID_ARG for
+ * unknown flag bits, a null strength or misaligned pointers, and the same
+ * dimension errors as gdr2_chunk_fwd. Asynchronous on `stream`.
+ */
+#define GDR2_QED_GATE 1u
+#define GDR2_QED_PROJECT 2u
+gdr2_status gdr2_qed_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const void *b, const void *w, const float *strength,
+                         const float *direction, uint32_t flags, const float *init_state,
+                         const int32_t *cu_seqlens, int64_t B, int64_t T, int64_t H,
+                         int64_t d_k, int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                         void *o, float *final_state, void *stream);
+
+/*
  * gdr2_check_device_error -- reports whether a kernel of this library gave up
  * a bounded device-side wait on the current device since the last check.
  *

@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                 _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int,
                 _vp, _vp, _vp]
+            L.gdr2_qed_fwd.restype = ctypes.c_int
+            L.gdr2_qed_fwd.argtypes = [
+                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_uint32, _vp, _vp,
+                _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_int, _vp, _vp, _vp]
             L.gdr2_check_device_error.restype = ctypes.c_int
             L.gdr2_check_device_error.argtypes = [_vp]
             L.gdr2_recurrent_step.restype = ctypes.c_int
@@ -314,6 +318,58 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, init_state=None, cu_seqlens=None
         _stream_handle(stream))
     if st != GDR2_OK:
         raise GDR2Error("gdr2_chunk_fwd_noalloc", st)
+    return o, final_state
+
+
+GDR2_QED_GATE = 1
+GDR2_QED_PROJECT = 2
+
+
+def qed_fwd(q, k, v, log_alpha, b, w, strength, direction=None,
+            flags: int = GDR2_QED_GATE | GDR2_QED_PROJECT, init_state=None, cu_seqlens=None, *,
+            o=None, final_state=None, output_final_state: bool = True,
+            stream=None) -> Tuple["torch.Tensor", Optional["torch.Tensor"]]:
+    """Forward with the QED second erase direction (gdr2_qed_fwd in gdr2.h; a
+    reading of a page that does not print the update). Inputs and outputs as
+    chunk_fwd, plus strength: fp32 [H] on the device, direction: fp32 [H, d_k]
+    or None (the query), flags: GDR2_QED_* bits."""
+    import torch
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("qed_fwd needs CUDA tensors")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t, d in (("k", k, dk), ("b", b, dk), ("v", v, dv), ("w", w, dv)):
+        _check(t, name, (B, T, H, d), dt, dev)
+    _check(q, "q", (B, T, H, dk), dt, dev)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    _check(strength, "strength", (H,), torch.float32, dev)
+    if direction is not None:
+        _check(direction, "direction", (H, dk), torch.float32, dev)
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+        N = cu_seqlens.shape[0] - 1
+    else:
+        N = B
+    if init_state is not None:
+        _check(init_state, "init_state", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _check(final_state, "final_state", (N, H, dk, dv), torch.float32, dev)
+    st = lib().gdr2_qed_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(strength), _ptr(direction),
+        int(flags), _ptr(init_state), _ptr(cu_seqlens), B, T, H, dk, dv, N, code, _ptr(o),
+        _ptr(final_state), _stream_handle(stream))
+    if st != GDR2_OK:
+        raise GDR2Error("gdr2_qed_fwd", st)
     return o, final_state
 
 

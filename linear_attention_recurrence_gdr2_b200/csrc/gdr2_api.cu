@@ -256,6 +256,51 @@ gdr2_status gdr2_recurrent_step_preact(const void *q, const void *k, const void 
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
+gdr2_status gdr2_qed_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const void *b, const void *w, const float *strength,
+                         const float *direction, uint32_t flags, const float *init_state,
+                         const int32_t *cu_seqlens, int64_t B, int64_t T, int64_t H,
+                         int64_t d_k, int64_t d_v, int64_t num_seqs, gdr2_dtype dtype,
+                         void *o, float *final_state, void *stream)
+{
+    if (flags & ~(GDR2_QED_GATE | GDR2_QED_PROJECT)) return GDR2_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_FP32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    gdr2_status st = check_dims(d_k, d_v);
+    if (st != GDR2_OK) return st;
+    if (cu_seqlens) {
+        if (B != 1) return GDR2_ERR_INVALID_ARG;
+    } else if (num_seqs != B) {
+        return GDR2_ERR_INVALID_ARG;
+    }
+    if (H > 65535 || num_seqs * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;
+    if (!strength || (reinterpret_cast<uintptr_t>(strength) & 3u)) return GDR2_ERR_INVALID_ARG;
+    if (direction && (reinterpret_cast<uintptr_t>(direction) & 3u)) return GDR2_ERR_INVALID_ARG;
+    if (B * T > 0) {
+        const void *ptrs[] = {q, k, v, log_alpha, b, w, o};
+        for (const void *p : ptrs)
+            if (!p || !aligned16(p)) return GDR2_ERR_INVALID_ARG;
+    }
+    if (init_state && !aligned16(init_state)) return GDR2_ERR_INVALID_ARG;
+    if (final_state && !aligned16(final_state)) return GDR2_ERR_INVALID_ARG;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDR2_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDR2_OK;
+    gdr2::QedArgs a;
+    a.q = q; a.k = k; a.v = v; a.b = b; a.w = w;
+    a.log_alpha = log_alpha;
+    a.strength = strength;
+    a.direction = direction;
+    a.flags = flags;
+    a.init_state = init_state;
+    a.cu_seqlens = cu_seqlens;
+    a.o = o;
+    a.final_state = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.num_seqs = num_seqs;
+    a.bf16 = dtype == GDR2_BF16;
+    cudaError_t e = gdr2::launch_qed(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
 gdr2_status gdr2_check_device_error(void *stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDR2_ERR_CUDA;

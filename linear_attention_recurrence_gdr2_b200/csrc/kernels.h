@@ -23,6 +23,21 @@ struct DecodeArgs {
     uint32_t pre = 0;          // GDR2_PROLOGUE_* flags applied on load
 };
 
+struct QedArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *log_alpha;
+    const float *strength;     // [H]
+    const float *direction;    // [H, dk] or null (the query)
+    uint32_t flags;            // GDR2_QED_*
+    const float *init_state;   // may be null
+    const int32_t *cu_seqlens; // may be null
+    void *o;
+    float *final_state;        // may be null
+    int64_t B, T, H, dk, dv, num_seqs;
+    bool bf16;
+};
+cudaError_t launch_qed(const QedArgs &a, cudaStream_t stream);
+
 struct ChunkArgs {
     const void *q, *k, *v, *b, *w;
     const float *log_alpha;

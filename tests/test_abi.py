@@ -195,3 +195,27 @@ def test_bwd_workspace_size():
 ])
 def test_chunk_bwd_rejects_bad_arguments(over, expect):
     assert _bwd(**over) == expect
+
+
+def _qed(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, lam=FAKE, dirs=None, flags=3, s0=None,
+             cu=None, B=2, T=64, H=4, dk=64, dv=64, N=2, dtype=0, o=FAKE, sf=None, stream=None)
+    a.update(over)
+    return gdr2.lib().gdr2_qed_fwd(a["q"], a["k"], a["v"], a["la"], a["b"], a["w"], a["lam"], a["dirs"],
+                                    a["flags"], a["s0"], a["cu"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                    a["N"], a["dtype"], a["o"], a["sf"], a["stream"])
+
+
+def test_qed_arguments_validated_on_the_host():
+    assert _qed(flags=4) == INVALID           # unknown flag bit
+    assert _qed(lam=None) == INVALID          # the strength is required
+    assert _qed(lam=FAKE + 2) == INVALID      # misaligned fp32 array
+    assert _qed(dirs=FAKE + 1) == INVALID
+    assert _qed(q=None) == INVALID
+    assert _qed(o=FAKE + 8) == INVALID        # token tensors 16-byte aligned
+    assert _qed(dk=96, dv=96) == UNSUPPORTED
+    assert _qed(dk=64, dv=128) == UNSUPPORTED
+    assert _qed(N=3) == INVALID               # num_seqs must equal B without cu_seqlens
+    assert _qed(cu=FAKE, B=2) == INVALID      # packed batches have B = 1
+    assert _qed(dtype=7) == INVALID
+    assert _qed(B=0, N=0, q=None, o=None) == OK

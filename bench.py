@@ -349,6 +349,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-qed", action="store_true")
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="skip the long-context and packed-batch objects")
     ap.add_argument("--extra-launches", type=int, default=4)
@@ -557,6 +558,24 @@ def main():
                    "peak_tflops": SIMT_FP32_TFLOPS, "frac": fl / (bms * 1e-3) / 1e12 / SIMT_FP32_TFLOPS,
                    "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz"}
 
+        # QED second erase direction on the same batch (a reading; token-serial CUDA-core path)
+        qed = None
+        if not args.no_qed:
+            log("qed")
+            lam = torch.full((H,), 0.1, dtype=torch.float32, device=dev)
+
+            def qstep():
+                return gdr2.qed_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["b"], t["w"], lam, None, 3,
+                                    t["s0"], t["cu"], o=t["o"], final_state=t["sf"])
+
+            qstep()
+            barrier()
+            qst = stats_ms(per_launch(qstep, 3))
+            qms = max_over_ranks(qst["median_us"]) * 1e-3
+            qed = {"kernel": "qed_fwd_kernel (token-serial, fp32 CUDA cores; strength 0.1, full arm)",
+                   "calls": 3, **qst, "tokens_per_s": inp.num_tokens / (qms * 1e-3),
+                   "note": "a reading of a page that does not print the update; parity unpinned"}
+
     ms_per_step = total_ms / args.steps
     value = aggregate_throughput(inp.num_tokens, world, ms_per_step)
     pst = stats_ms(per)
@@ -601,6 +620,8 @@ def main():
         line["e2e"] = e2e
     if bwd is not None:
         line["backward"] = bwd
+    if qed is not None:
+        line["qed"] = qed
     if world == 1 and not args.no_cpu_baseline:
         log("cpu baseline")
         line["cpu_baseline"] = cpu_baseline(inp, label)

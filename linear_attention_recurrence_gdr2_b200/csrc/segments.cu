@@ -59,10 +59,21 @@ seg_combine_kernel(float *__restrict__ s0, const float *__restrict__ phi, float 
     const int64_t h = blockIdx.y, n = blockIdx.z;
     const int r0 = kCombRows * (int)blockIdx.x;
     auto slot = [&](int q) { return ((n * nseg + q) * H + h) * kStateElems; };
+    // (all loads of a thread are issued before its first store, so their
+    // latencies overlap)
     const float4 *src = reinterpret_cast<const float4 *>(s0 + slot(p - 1));
-    for (int i = tid; i < (int)(kStateElems / 4); i += 256) comb4[i] = src[i];
     const float4 *prow = reinterpret_cast<const float4 *>(phi + slot(p) + (int64_t)r0 * kD);
-    for (int i = tid; i < kCombRows * kD / 4; i += 256) comb4[kStateElems / 4 + i] = prow[i];
+    {
+        float4 x[kStateElems / 4 / 256], y[kCombRows * kD / 4 / 256];
+#pragma unroll
+        for (int i = 0; i < (int)(kStateElems / 4 / 256); ++i) x[i] = src[tid + 256 * i];
+#pragma unroll
+        for (int i = 0; i < kCombRows * kD / 4 / 256; ++i) y[i] = prow[tid + 256 * i];
+#pragma unroll
+        for (int i = 0; i < (int)(kStateElems / 4 / 256); ++i) comb4[tid + 256 * i] = x[i];
+#pragma unroll
+        for (int i = 0; i < kCombRows * kD / 4 / 256; ++i) comb4[kStateElems / 4 + tid + 256 * i] = y[i];
+    }
     __syncthreads();
     const int rr = tid >> 4, c8 = 8 * (tid & 15);
     const float *s0r = s0 + slot(p) + (int64_t)(r0 + rr) * kD + c8;
@@ -95,11 +106,13 @@ seg_combine_kernel(float *__restrict__ s0, const float *__restrict__ phi, float 
 // (the product keeps about 16 mantissa bits of S). One CTA stages S once and
 // runs up to kCorrTiles tiles of one
 // (sequence, head): warp 0 loads Psi tiles by TMA (two slots), warp 1 issues
-// the 16 MMAs of a tile into one of two TMEM accumulators, warps 4-7 add the
-// accumulator to o (thread = token row = TMEM lane). Every wait is bounded.
+// the 16 MMAs of a tile into one of two TMEM accumulators, warps 4-11 add the
+// accumulator to o (thread = token row = TMEM lane, two warps per lane quarter
+// taking 64 output channels each), loading the next tile's o rows before they
+// work on the current one. Every wait is bounded.
 constexpr int kCorrRows = 128;     // tokens per tile (the MMA's M)
 constexpr int kCorrTiles = 16;     // tiles per CTA: S^T is staged once per 2048 tokens
-constexpr int kCorrThreads = 256;
+constexpr int kCorrThreads = 384;  // warp 0 TMA, warp 1 MMA, warp 2 TMEM, warps 4-11 epilogue
 constexpr uint32_t kCB = 0;        // S [part hi, lo][j half][128 k rows x 128 B], 64 KB
 constexpr uint32_t kCA = 65536;    // Psi slots [2][k half][128 rows x 128 B], 32 KB each
 constexpr uint32_t kCBar = 131072;
@@ -155,9 +168,19 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
     // layout: rows k, 64 output channels per 128-byte row, channel halves apart
     {
         const float4 *src = reinterpret_cast<const float4 *>(sst + ((n * nseg + p - 1) * H + h) * kStateElems);
-        for (int i = tid; i < (int)(kStateElems / 4); i += kCorrThreads) {
+        constexpr int kPer = (int)((kStateElems / 4 + kCorrThreads - 1) / kCorrThreads);
+        float4 xin[kPer];
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {  // (every load before the first store)
+            const int i = tid + kCorrThreads * m;
+            if (i < (int)(kStateElems / 4)) xin[m] = src[i];
+        }
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+            const int i = tid + kCorrThreads * m;
+            if (i >= (int)(kStateElems / 4)) break;
             const int k = i >> 5, j = 4 * (i & 31);
-            const float4 x = src[i];
+            const float4 x = xin[m];
             const float xs[4] = {x.x, x.y, x.z, x.w};
             uint32_t hi[2], lo[2];
 #pragma unroll
@@ -235,39 +258,56 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
             mbar_wait(&bars[C_DRAIN], 0, g, 44);
         }
     } else if (warp >= 4) {
-        // ---- o rows += D rows (thread = token row = TMEM lane) ----
-        const int q4 = warp & 3, row = 32 * q4 + lane, te = tid - 128;
+        // ---- o rows += D rows (thread = token row = TMEM lane; 64 channels) ----
+        const int q4 = warp & 3, half = (warp - 4) >> 2, row = 32 * q4 + lane, te = tid - 128;
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        auto orow = [&](int i) -> uint4 * {
+            const int64_t t = tb + (int64_t)kCorrRows * i + row;
+            return reinterpret_cast<uint4 *>(o + ((n * T + t) * H + h) * kD + 64 * half);
+        };
+        auto in_seg = [&](int i) { return tb + (int64_t)kCorrRows * i + row < seg_end; };
+        uint4 cur[8], nxt[8];
+        if (in_seg(0)) {
+            const uint4 *po = orow(0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cur[e] = po[e];
+        }
         for (int i = 0; i < ntiles; ++i) {
             const int s = i & 1;
-            if (!group_all(kBarEpiC, 128, cwait(&bars[C_ACC0 + s], (i >> 1) & 1, abort_flag, 45))) break;
+            if (!group_all(kBarEpiC, 256, cwait(&bars[C_ACC0 + s], (i >> 1) & 1, abort_flag, 45))) break;
             tc_fence_after();
-            const int64_t t = tb + (int64_t)kCorrRows * i + row;
-            __nv_bfloat16 *orow = o + ((n * T + t) * H + h) * kD;
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
+            if (i + 1 < ntiles && in_seg(i + 1)) {  // the next tile's rows, while this one is added
+                const uint4 *pn = orow(i + 1);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) nxt[e] = pn[e];
+            }
+            const bool mine = in_seg(i);
+            uint4 *po = orow(i);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
                 uint32_t v[32];
-                tmem_ld32(tbase + 128 * s + 32 * q + lane_off, v);
+                tmem_ld32(tbase + 128 * s + 64 * half + 32 * qq + lane_off, v);
                 tc_wait_ld();
-                if (t < seg_end) {
-                    uint4 *po = reinterpret_cast<uint4 *>(orow + 32 * q);
+                if (mine) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        uint4 x = po[e];
-                        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                        const uint4 x = cur[4 * qq + e];
+                        uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[c]));
-                            w[c] = pack_bf16x2(f.x + __uint_as_float(v[8 * e + 2 * c]),
-                                               f.y + __uint_as_float(v[8 * e + 2 * c + 1]));
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w4[c]));
+                            w4[c] = pack_bf16x2(f.x + __uint_as_float(v[8 * e + 2 * c]),
+                                                f.y + __uint_as_float(v[8 * e + 2 * c + 1]));
                         }
-                        po[e] = make_uint4(w[0], w[1], w[2], w[3]);
+                        po[4 * qq + e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
             }
             tc_fence_before();
-            named_bar_sync(kBarEpiC, 128);
+            named_bar_sync(kBarEpiC, 256);
             if (te == 0) mbar_arrive(&bars[C_ACCFREE0 + s]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cur[e] = nxt[e];
         }
     }
     tc_fence_before();

@@ -23,8 +23,9 @@
 //     decay sums and factors Qm, Km, Em (in place over the q, k, b tiles),
 //     [A^T | P^T] = Km [Em; Qm]^T       M=64  N=128 K=128 (tcgen05),
 //     T = (I + A)^{-1} (tf32 mma.sync doubling) as bf16,
-//     and bulk copies of Em, Qm, Km, P^T, T and the half sums into the main
-//     CTA's shared memory (distributed shared memory inside the cluster);
+//     bulk copies of Em, Qm, Km, P^T and the half sums, and remote 16-byte
+//     stores of T, into the main CTA's shared memory (distributed shared
+//     memory inside the cluster);
 //   main CTA (cluster ranks 0, 1), per chunk:
 //     Z = w . v; -W = -(T Em) (two M=64 halves); U0^T = Z^T T^T;
 //     [U^T | O^T]  += Sm^T [-W; Qm]^T   M=128 N=128 K=128, A in TMEM

@@ -78,3 +78,15 @@ def test_qed_zero_strength_matches_the_chunk_forward(cuda_device):
     torch.cuda.synchronize()
     assert_close("qed strength 0 vs chunk forward", o, to_np(o_c), "fp32")
     assert_close("qed strength 0 state vs chunk forward", sf, to_np(sf_c), "fp32")
+
+
+def test_qed_query_parallel_to_key_is_the_plain_rule(cuda_device):
+    """Degenerate case of the reading: a query parallel to the key has no part
+    orthogonal to it, so the second erase vanishes and the step is the plain
+    rule (both sides decide u = 0 by the same relative threshold)."""
+    inp = gen.make_inputs(1, 90, 2, 64, 64, "fp32", seed=56, init_std=0.05)
+    inp.q[...] = 2.0 * inp.k
+    o, sf, _, _ = run(inp, cuda_device, [0.7, 1.0])
+    o_p, sf_p = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.b, inp.w, inp.init_state)
+    assert_close("qed q || k o", o, o_p, "fp32")
+    assert_close("qed q || k state", sf, sf_p, "fp32")

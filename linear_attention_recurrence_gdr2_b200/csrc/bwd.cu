@@ -82,14 +82,15 @@ __device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16 *p, float a,
     *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
 }
 
-// ROWS consecutive floats from shared memory (16-byte aligned) as float4 loads.
-template <int ROWS>
-__device__ __forceinline__ void load_rows(const float *src, float (&out)[ROWS])
+// ROWS floats from shared memory in groups of 4: group g at src + g * GS (each
+// group one 16-byte load).
+template <int ROWS, int GS>
+__device__ __forceinline__ void load_row_groups(const float *src, float (&out)[ROWS])
 {
     static_assert(ROWS % 4 == 0, "rows come in float4 groups");
 #pragma unroll
     for (int g = 0; g < ROWS / 4; ++g) {
-        const float4 v = *reinterpret_cast<const float4 *>(src + 4 * g);
+        const float4 v = *reinterpret_cast<const float4 *>(src + GS * g);
         out[4 * g] = v.x; out[4 * g + 1] = v.y; out[4 * g + 2] = v.z; out[4 * g + 3] = v.w;
     }
 }
@@ -107,8 +108,9 @@ __device__ __forceinline__ void cp_async_wait_all()
 
 // Sweeps A (blockIdx.z == 0) and B (blockIdx.z == 1). CTA = (sequence, head,
 // tile of 64 value columns); lane l of warp w owns the 4 columns 64*tile + 8w +
-// 4*(l/16) + {0..3} and the D/16 consecutive key rows starting at (l % 16) *
-// D/16 (read from shared memory as float4), so the reductions over key rows are
+// 4*(l/16) + {0..3} and D/16 key rows in groups of 4 (group g: rows
+// 64 g + 4 (l % 16) + {0..3}, read from shared memory as float4 without bank
+// conflicts), so the reductions over key rows are
 // four xor-shuffles inside a half-warp, four independent columns at a time. One
 // CTA per 64 columns keeps both sweeps of a layer-sized batch resident at once.
 // Row inputs (alpha, e, k, q) for 8 tokens are staged in shared memory, the
@@ -130,7 +132,12 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     const int tile = blockIdx.y;
     const bool rev = blockIdx.z != 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row0 = (lane & 15) * ROWS;            // first of this lane's key rows
+    // this lane's key rows: ROWS/4 groups of 4, group g at g * GS + 4 (lane % 16),
+    // so that the 16 lanes' 16-byte reads of one group are one contiguous 256 B
+    // (no shared-memory bank conflicts)
+    constexpr int GS = D / (ROWS / 4);
+    const int row0 = 4 * (lane & 15);
+    auto row_of = [&](int m) { return GS * (m >> 2) + row0 + (m & 3); };
     const int jl = warp * 2 * NC + (lane >> 4) * NC;  // first of this lane's columns, in the tile
     const int j = tile * kTile + jl;
     const Tin *Q = static_cast<const Tin *>(p.q), *K = static_cast<const Tin *>(p.k);
@@ -143,13 +150,13 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     const int64_t nsub = (len + kSub - 1) / kSub;
     const int64_t head_state = (n * p.H + h) * (int64_t)D * D;
 
-    // X: state columns (A) or cotangent columns (B), rows row0 .. row0 + ROWS - 1
+    // X: state columns (A) or cotangent columns (B), rows row_of(0 .. ROWS - 1)
     float X[NC][ROWS];
     const float *x_init = rev ? p.d_final : p.init_state;
 #pragma unroll
     for (int m = 0; m < ROWS; ++m) {
         float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (x_init) v4 = *reinterpret_cast<const float4 *>(x_init + head_state + (int64_t)(row0 + m) * D + j);
+        if (x_init) v4 = *reinterpret_cast<const float4 *>(x_init + head_state + (int64_t)row_of(m) * D + j);
         X[0][m] = v4.x; X[1][m] = v4.y; X[2][m] = v4.z; X[3][m] = v4.w;
     }
 
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
             float *dst = (rev ? p.gk : p.ck) + ((base + chunk) * p.H + h) * (int64_t)D * D;
 #pragma unroll
             for (int m = 0; m < ROWS; ++m)
-                *reinterpret_cast<float4 *>(dst + (int64_t)(row0 + m) * D + j) =
+                *reinterpret_cast<float4 *>(dst + (int64_t)row_of(m) * D + j) =
                     make_float4(X[0][m], X[1][m], X[2][m], X[3][m]);
         }
 
@@ -228,9 +235,9 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
             for (int tt = 0; tt < L; ++tt) {
                 const int64_t tok = start + sb * kSub + tt;
                 float r[NC] = {0.f, 0.f, 0.f, 0.f}, al[ROWS], ee[ROWS], kk[ROWS];
-                load_rows<ROWS>(s_al + tt * D + row0, al);
-                load_rows<ROWS>(s_e + tt * D + row0, ee);
-                load_rows<ROWS>(s_k + tt * D + row0, kk);
+                load_row_groups<ROWS, GS>(s_al + tt * D + row0, al);
+                load_row_groups<ROWS, GS>(s_e + tt * D + row0, ee);
+                load_row_groups<ROWS, GS>(s_k + tt * D + row0, kk);
 #pragma unroll
                 for (int m = 0; m < ROWS; ++m)
 #pragma unroll
@@ -258,10 +265,10 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
                 const float4 o4 = *reinterpret_cast<const float4 *>(&s_c[0][cb]);
                 const float oo[NC] = {o4.x, o4.y, o4.z, o4.w};
                 float d[NC] = {0.f, 0.f, 0.f, 0.f}, qq[ROWS], kk[ROWS], al[ROWS], ee[ROWS];
-                load_rows<ROWS>(s_q + tt * D + row0, qq);
-                load_rows<ROWS>(s_k + tt * D + row0, kk);
-                load_rows<ROWS>(s_al + tt * D + row0, al);
-                load_rows<ROWS>(s_e + tt * D + row0, ee);
+                load_row_groups<ROWS, GS>(s_q + tt * D + row0, qq);
+                load_row_groups<ROWS, GS>(s_k + tt * D + row0, kk);
+                load_row_groups<ROWS, GS>(s_al + tt * D + row0, al);
+                load_row_groups<ROWS, GS>(s_e + tt * D + row0, ee);
 #pragma unroll
                 for (int m = 0; m < ROWS; ++m)
 #pragma unroll
@@ -294,7 +301,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) bwd_scan_kernel(BwdParams p)
     if (rev && p.d_init) {
 #pragma unroll
         for (int m = 0; m < ROWS; ++m)
-            *reinterpret_cast<float4 *>(p.d_init + head_state + (int64_t)(row0 + m) * D + j) =
+            *reinterpret_cast<float4 *>(p.d_init + head_state + (int64_t)row_of(m) * D + j) =
                 make_float4(X[0][m], X[1][m], X[2][m], X[3][m]);
     }
 }

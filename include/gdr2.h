@@ -355,11 +355,12 @@ gdr2_status gdr2_qed_fwd(const void *q, const void *k, const void *v, const floa
  * gdr2_check_device_error -- reports whether a kernel of this library gave up
  * a bounded device-side wait on the current device since the last check.
  *
- * The tensor-core chunk kernel bounds every wait inside the GPU (about one
- * second without progress); when one runs out, the affected CTA records the
- * site in a device-global error word, drains its in-flight copies and MMAs,
- * frees its tensor memory and returns, leaving its outputs incomplete. This
- * call synchronises `stream`, then reads and clears that word. Returns
+ * The tensor-core kernels (the chunk forward and the segment split's output
+ * correction) bound every wait inside the GPU (about one second without
+ * progress); when one runs out, the affected CTA records the site in a
+ * device-global error word, drains its in-flight copies and MMAs, frees its
+ * tensor memory and returns, leaving its outputs incomplete. This call
+ * synchronises `stream`, then reads and clears those words. Returns
  * GDR2_OK (no timeout), GDR2_ERR_DEVICE_TIMEOUT, or GDR2_ERR_CUDA if the
  * synchronisation or the read failed.
  */

@@ -104,14 +104,14 @@ seg_combine_kernel(float *__restrict__ s0, const float *__restrict__ phi, float 
 // staged as the MMA's B operand in its MN-major layout (rows k, output
 // channels contiguous, as S is stored); both parts accumulate into the same D
 // (the product keeps about 16 mantissa bits of S). One CTA stages S once and
-// runs up to kCorrTiles tiles of one
-// (sequence, head): warp 0 loads Psi tiles by TMA (two slots), warp 1 issues
+// runs up to kCorrTiles tiles of one (sequence, head): warp 0 loads Psi tiles
+// by TMA (two slots), warp 1 issues
 // the 16 MMAs of a tile into one of two TMEM accumulators, warps 4-11 add the
 // accumulator to o (thread = token row = TMEM lane, two warps per lane quarter
 // taking 64 output channels each), loading the next tile's o rows before they
 // work on the current one. Every wait is bounded.
 constexpr int kCorrRows = 128;     // tokens per tile (the MMA's M)
-constexpr int kCorrTiles = 16;     // tiles per CTA: S^T is staged once per 2048 tokens
+constexpr int kCorrTiles = 16;     // tiles per CTA: S is staged once per 2048 tokens
 constexpr int kCorrThreads = 384;  // warp 0 TMA, warp 1 MMA, warp 2 TMEM, warps 4-11 epilogue
 constexpr uint32_t kCB = 0;        // S [part hi, lo][j half][128 k rows x 128 B], 64 KB
 constexpr uint32_t kCA = 65536;    // Psi slots [2][k half][128 rows x 128 B], 32 KB each

@@ -108,14 +108,16 @@ seg_combine_kernel(float *__restrict__ s0, const float *__restrict__ phi, float 
 // by TMA (two slots), warp 1 issues
 // the 16 MMAs of a tile into one of two TMEM accumulators, warps 4-11 add the
 // accumulator to o (thread = token row = TMEM lane, two warps per lane quarter
-// taking 64 output channels each), loading the next tile's o rows before they
-// work on the current one. Every wait is bounded.
+// taking 64 output channels each). The tile's o rows arrive by TMA with its
+// Psi rows, so the epilogue reads them from shared memory and only stores to
+// global memory. Every wait is bounded.
 constexpr int kCorrRows = 128;     // tokens per tile (the MMA's M)
 constexpr int kCorrTiles = 16;     // tiles per CTA: S is staged once per 2048 tokens
 constexpr int kCorrThreads = 384;  // warp 0 TMA, warp 1 MMA, warp 2 TMEM, warps 4-11 epilogue
 constexpr uint32_t kCB = 0;        // S [part hi, lo][j half][128 k rows x 128 B], 64 KB
 constexpr uint32_t kCA = 65536;    // Psi slots [2][k half][128 rows x 128 B], 32 KB each
-constexpr uint32_t kCBar = 131072;
+constexpr uint32_t kCO = 131072;   // o slots, the same layout (channel halves apart)
+constexpr uint32_t kCBar = 196608;
 enum { C_FULL0 = 0, C_FULL1, C_FREE0, C_FREE1, C_ACC0, C_ACC1, C_ACCFREE0, C_ACCFREE1, C_DRAIN, C_NUM };
 constexpr uint32_t kCMisc = kCBar + C_NUM * 8;      // TMEM base, abort flag
 constexpr uint32_t kCorrSmem = kCMisc + 16 + 1024;  // + alignment slack
@@ -144,7 +146,8 @@ __device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
 }
 
 __global__ void __launch_bounds__(kCorrThreads, 1)
-seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *__restrict__ o,
+seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, const __grid_constant__ CUtensorMap map_o,
+                   __nv_bfloat16 *__restrict__ o,
                    const float *__restrict__ sst, int nseg, int64_t seg_len, int64_t T, int64_t H)
 {
     using namespace sm100;
@@ -197,10 +200,15 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
     }
     if (tid == 0) {
         for (int i = 0; i < C_NUM; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&bars[C_FREE0], 2);  // a slot is free once its MMAs and its o readers are done
+        mbar_init(&bars[C_FREE1], 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) prefetch_tensormap(&map_psi);
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&map_psi);
+        prefetch_tensormap(&map_o);
+    }
     if (warp == 2) {
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
@@ -211,17 +219,20 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
     const uint32_t tbase = *tmem_slot;
 
     if (warp == 0) {
-        // ---- Psi tiles by TMA (two slots) ----
+        // ---- Psi and o tiles by TMA (two slots) ----
         if (lane == 0) {
             int issued0 = 0, issued1 = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i & 1;
                 if (i >= 2 && !cwait(&bars[C_FREE0 + s], ((i >> 1) - 1) & 1, abort_flag, 40)) break;
                 const int z = (int)(n * T + tb + (int64_t)kCorrRows * i);
-                mbar_arrive_expect_tx(&bars[C_FULL0 + s], 32768);
-                for (int half = 0; half < 2; ++half)
+                mbar_arrive_expect_tx(&bars[C_FULL0 + s], 65536);
+                for (int half = 0; half < 2; ++half) {
                     tma_load_3d(smem + kCA + s * 32768 + half * 16384, &map_psi, &bars[C_FULL0 + s], 64 * half,
                                 (int)h, z);
+                    tma_load_3d(smem + kCO + s * 32768 + half * 16384, &map_o, &bars[C_FULL0 + s], 64 * half,
+                                (int)h, z);
+                }
                 (s ? issued1 : issued0) = (i >> 1) + 1;
             }
             // (loads still in flight after an abort land before the CTA exits)
@@ -261,28 +272,17 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
         // ---- o rows += D rows (thread = token row = TMEM lane; 64 channels) ----
         const int q4 = warp & 3, half = (warp - 4) >> 2, row = 32 * q4 + lane, te = tid - 128;
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        auto orow = [&](int i) -> uint4 * {
-            const int64_t t = tb + (int64_t)kCorrRows * i + row;
-            return reinterpret_cast<uint4 *>(o + ((n * T + t) * H + h) * kD + 64 * half);
-        };
-        auto in_seg = [&](int i) { return tb + (int64_t)kCorrRows * i + row < seg_end; };
-        uint4 cur[8], nxt[8];
-        if (in_seg(0)) {
-            const uint4 *po = orow(0);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) cur[e] = po[e];
-        }
         for (int i = 0; i < ntiles; ++i) {
             const int s = i & 1;
-            if (!group_all(kBarEpiC, 256, cwait(&bars[C_ACC0 + s], (i >> 1) & 1, abort_flag, 45))) break;
+            // (the FULL wait makes the TMA-written o rows visible to these threads)
+            if (!group_all(kBarEpiC, 256, cwait(&bars[C_ACC0 + s], (i >> 1) & 1, abort_flag, 45) &&
+                                              cwait(&bars[C_FULL0 + s], (i >> 1) & 1, abort_flag, 46)))
+                break;
             tc_fence_after();
-            if (i + 1 < ntiles && in_seg(i + 1)) {  // the next tile's rows, while this one is added
-                const uint4 *pn = orow(i + 1);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) nxt[e] = pn[e];
-            }
-            const bool mine = in_seg(i);
-            uint4 *po = orow(i);
+            const int64_t t = tb + (int64_t)kCorrRows * i + row;
+            const bool mine = t < seg_end;
+            uint4 *po = reinterpret_cast<uint4 *>(o + ((n * T + t) * H + h) * kD + 64 * half);
+            const unsigned char *so = smem + kCO + s * 32768 + half * 16384;
 #pragma unroll
             for (int qq = 0; qq < 2; ++qq) {
                 uint32_t v[32];
@@ -291,7 +291,7 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
                 if (mine) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const uint4 x = cur[4 * qq + e];
+                        const uint4 x = *reinterpret_cast<const uint4 *>(so + sw128_offset(row, 16 * (4 * qq + e)));
                         uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -305,9 +305,10 @@ seg_correct_kernel(const __grid_constant__ CUtensorMap map_psi, __nv_bfloat16 *_
             }
             tc_fence_before();
             named_bar_sync(kBarEpiC, 256);
-            if (te == 0) mbar_arrive(&bars[C_ACCFREE0 + s]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) cur[e] = nxt[e];
+            if (te == 0) {
+                mbar_arrive(&bars[C_ACCFREE0 + s]);
+                mbar_arrive(&bars[C_FREE0 + s]);  // (its o rows have been read)
+            }
         }
     }
     tc_fence_before();
@@ -395,8 +396,12 @@ cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream)
     cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)(a.H * kD * 2)};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)kCorrRows};
     cuuint32_t es[3] = {1, 1, 1};
+    CUtensorMap map_o;  // o, the same shape and box
     if (enc(&map_psi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(psi), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        enc(&map_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.o, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     e = ensure_dynamic_smem((const void *)seg_correct_kernel, (int)kCorrSmem);
@@ -404,7 +409,7 @@ cudaError_t launch_segment_fix(const ChunkArgs &a, cudaStream_t stream)
     const int64_t per_seg = (a.seg_len + kCorrRows * kCorrTiles - 1) / (kCorrRows * kCorrTiles);
     const int64_t nblk = per_seg * (a.nseg - 1);  // segments 1..nseg-1
     dim3 grid((unsigned)nblk, (unsigned)a.H, (unsigned)a.B);
-    seg_correct_kernel<<<grid, kCorrThreads, kCorrSmem, stream>>>(map_psi, static_cast<__nv_bfloat16 *>(a.o), s0,
+    seg_correct_kernel<<<grid, kCorrThreads, kCorrSmem, stream>>>(map_psi, map_o, static_cast<__nv_bfloat16 *>(a.o), s0,
                                                                  a.nseg, a.seg_len, a.T, a.H);
     return cudaGetLastError();
 }

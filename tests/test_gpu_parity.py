@@ -166,6 +166,8 @@ def test_chunk_strong_decay_in_range(cuda_device):
     (1, 2048, 2, 0.01, 0.05),    # 4 segments of 512 tokens, nonzero initial state
     (2, 1000, 3, 0.02, None),    # 2 segments, ragged last chunk
     (1, 8192, 1, 0.005, 0.02),   # 16 segments: the longest combine chain
+    (1, 1700, 1, 0.02, 0.05),    # 3 segments of 576 tokens: correction tiles of 128 rows
+                                 # straddle the segment boundaries; ragged end
 ])
 def test_chunk_segment_split(cuda_device, B, T, H, la_scale, init):
     """Few long bf16 sequences run as concurrent segments (from the segment's

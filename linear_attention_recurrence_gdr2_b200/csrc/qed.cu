@@ -15,9 +15,11 @@
 // head, 32 value columns) runs the tokens in order. Columns of S evolve
 // independently given k, u, b and alpha, so the value blocks of one head need
 // no communication. Thread (warp w, lane l) keeps rows w*DK/4 .. of column l
-// in registers; each token costs three block reductions (the direction's
-// norms, the two reads of the decayed state, the readout), and its inputs are
-// loaded one token ahead.
+// in registers. Every warp computes the token's direction u on its own (warp
+// shuffles over the DK channels, lane l holding channels l + 32m) and keeps the
+// per-channel factors in its own shared-memory slice, so a token costs two
+// block barriers (the two reads of the decayed state, then the readout, summed
+// over the warps); its inputs are loaded one token ahead.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,10 +38,12 @@ qed_fwd_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *
                const float *__restrict__ init_state, const int32_t *__restrict__ cu_seqlens, int64_t T,
                int64_t H, int64_t DV, int64_t tokens, Tin *__restrict__ o, float *__restrict__ final_state)
 {
-    constexpr int ROWS = DK / 4;  // key rows per warp
-    __shared__ float s_q[DK], s_k[DK], s_a[DK], s_e[DK], s_u[DK], s_f[DK];
-    __shared__ float s_red[4][3];
-    __shared__ float s_rk[4][kQedCols], s_ru[4][kQedCols];
+    constexpr int ROWS = DK / 4;   // key rows per warp
+    constexpr int CPL = DK / 32;   // channels per lane in the direction's reductions
+    // per warp: alpha, e = b . k, k, u, f, q for every channel (written and read
+    // by the same warp only)
+    __shared__ float s_v[4][6][DK];
+    __shared__ float s_rk[4][kQedCols], s_ru[4][kQedCols], s_o[4][kQedCols];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t unit = blockIdx.x, n = unit / H, h = unit % H;
@@ -53,79 +57,91 @@ qed_fwd_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *
     }
     const float lambda = strength[h];
     const bool gate = (flags & GDR2_QED_GATE) != 0, project = (flags & GDR2_QED_PROJECT) != 0;
-    const float dirc = (direction && tid < DK) ? direction[h * DK + tid] : 0.f;
+    float dirc[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) dirc[m] = direction ? direction[h * DK + lane + 32 * m] : 0.f;
 
     float s[ROWS];
     const int64_t sbase = (unit * DK + (int64_t)ROWS * warp) * DV + j;
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) s[i] = init_state ? init_state[sbase + (int64_t)i * DV] : 0.f;
 
-    // block sum of three values (one per thread; the result in every thread)
-    auto sum3 = [&](float &x, float &y, float &z) {
+    auto warp_sum = [&](float x) {
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-            x += __shfl_xor_sync(0xffffffffu, x, m);
-            y += __shfl_xor_sync(0xffffffffu, y, m);
-            z += __shfl_xor_sync(0xffffffffu, z, m);
-        }
-        if (lane == 0) {
-            s_red[warp][0] = x;
-            s_red[warp][1] = y;
-            s_red[warp][2] = z;
-        }
-        __syncthreads();
-        x = s_red[0][0] + s_red[1][0] + s_red[2][0] + s_red[3][0];
-        y = s_red[0][1] + s_red[1][1] + s_red[2][1] + s_red[3][1];
-        z = s_red[0][2] + s_red[1][2] + s_red[2][2] + s_red[3][2];
-        __syncthreads();  // (s_red is reused by the next call)
+        for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+        return x;
     };
 
-    // inputs of token t: channel tid (tid < DK) of q, k, log_alpha, b; value
-    // column j of v and w (every warp loads the same 32 columns)
-    float nq = 0.f, nk = 0.f, nla = 0.f, nb = 0.f, nv = 0.f, nw = 0.f;
+    // inputs of token t: channels lane + 32m of q, k, log_alpha, b; value
+    // column j of v and w
+    float nq[CPL], nk[CPL], nla[CPL], nb[CPL], nv = 0.f, nw = 0.f;
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) nq[m] = nk[m] = nla[m] = nb[m] = 0.f;
     auto fetch = [&](int64_t t) {
         if (t >= t_end) return;
         const int64_t rk = (t * H + h) * DK, rv = (t * H + h) * DV;
-        if (tid < DK) {
-            nq = to_f32(q[rk + tid]);
-            nk = to_f32(k[rk + tid]);
-            nla = log_alpha[rk + tid];
-            nb = to_f32(b[rk + tid]);
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            const int c = lane + 32 * m;
+            nq[m] = to_f32(q[rk + c]);
+            nk[m] = to_f32(k[rk + c]);
+            nla[m] = log_alpha[rk + c];
+            nb[m] = to_f32(b[rk + c]);
         }
         nv = to_f32(v[rv + j]);
         nw = to_f32(w[rv + j]);
     };
     fetch(t_begin);
+    float (&sv)[6][DK] = s_v[warp];
     for (int64_t t = t_begin; t < t_end; ++t) {
-        const float qc = nq, kc = nk, lac = nla, bc = nb, z = nv * nw;
-        fetch(t + 1);
-        // the erase direction u from the query (or the fixed direction)
-        const float src = direction ? dirc : qc;
-        float kk = tid < DK ? kc * kc : 0.f, ks = tid < DK ? kc * src : 0.f, ss = tid < DK ? src * src : 0.f;
-        sum3(kk, ks, ss);
-        const float coef = (project && kk > 0.f) ? ks / kk : 0.f;
-        const float pc = src - coef * kc;
-        float pp = tid < DK ? pc * pc : 0.f, d1 = 0.f, d2 = 0.f;
-        sum3(pp, d1, d2);
-        const float inv = (pp > 1e-12f * ss && pp > 0.f) ? rsqrtf(pp) : 0.f;
-        if (tid < DK) {
-            const float uc = pc * inv;
-            s_q[tid] = qc;
-            s_k[tid] = kc;
-            s_a[tid] = expf(lac);
-            s_e[tid] = bc * kc;
-            s_u[tid] = uc;
-            s_f[tid] = gate ? bc * uc : uc;
+        float qc[CPL], kc[CPL], lac[CPL], bc[CPL];
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            qc[m] = nq[m]; kc[m] = nk[m]; lac[m] = nla[m]; bc[m] = nb[m];
         }
-        __syncthreads();
+        const float z = nv * nw;
+        fetch(t + 1);
+        // the erase direction u from the query (or the fixed direction), in this warp
+        float kk = 0.f, ks = 0.f, ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            const float src = direction ? dirc[m] : qc[m];
+            kk = fmaf(kc[m], kc[m], kk);
+            ks = fmaf(kc[m], src, ks);
+            ss = fmaf(src, src, ss);
+        }
+        kk = warp_sum(kk);
+        ks = warp_sum(ks);
+        ss = warp_sum(ss);
+        const float coef = (project && kk > 0.f) ? ks / kk : 0.f;
+        float pc[CPL], pp = 0.f;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            pc[m] = (direction ? dirc[m] : qc[m]) - coef * kc[m];
+            pp = fmaf(pc[m], pc[m], pp);
+        }
+        pp = warp_sum(pp);
+        const float inv = (pp > 1e-12f * ss && pp > 0.f) ? rsqrtf(pp) : 0.f;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            const int c = lane + 32 * m;
+            const float uc = pc[m] * inv;
+            sv[0][c] = expf(lac[m]);
+            sv[1][c] = bc[m] * kc[m];
+            sv[2][c] = kc[m];
+            sv[3][c] = uc;
+            sv[4][c] = gate ? bc[m] * uc : uc;
+            sv[5][c] = qc[m];
+        }
+        __syncwarp();
         // decay, then both reads of the decayed state (this warp's rows)
         float rk = 0.f, ru = 0.f;
 #pragma unroll
         for (int i = 0; i < ROWS; ++i) {
             const int c = ROWS * warp + i;
-            s[i] *= s_a[c];
-            rk = fmaf(s_e[c], s[i], rk);
-            ru = fmaf(s_f[c], s[i], ru);
+            s[i] *= sv[0][c];
+            rk = fmaf(sv[1][c], s[i], rk);
+            ru = fmaf(sv[4][c], s[i], ru);
         }
         s_rk[warp][lane] = rk;
         s_ru[warp][lane] = ru;
@@ -138,17 +154,21 @@ qed_fwd_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *
 #pragma unroll
         for (int i = 0; i < ROWS; ++i) {
             const int c = ROWS * warp + i;
-            s[i] = fmaf(s_k[c], resid, fmaf(-s_u[c], lru, s[i]));
-            oq = fmaf(s_q[c], s[i], oq);
+            s[i] = fmaf(sv[2][c], resid, fmaf(-sv[3][c], lru, s[i]));
+            oq = fmaf(sv[5][c], s[i], oq);
         }
-        __syncthreads();  // (every read of s_rk / s_ru above is done)
-        s_rk[warp][lane] = oq;
+        s_o[warp][lane] = oq;
+        // (every thread has read s_rk / s_ru before it passes this barrier, and
+        // the next token writes them only after it)
         __syncthreads();
         if (warp == 0) {
-            const float oj = s_rk[0][lane] + s_rk[1][lane] + s_rk[2][lane] + s_rk[3][lane];
+            const float oj = s_o[0][lane] + s_o[1][lane] + s_o[2][lane] + s_o[3][lane];
             o[(t * H + h) * DV + j] = from_f32<Tin>(oj);
         }
-        // (the next token's first barrier orders these reads before s_rk is rewritten)
+        // (warp 0's reads of s_o come before its next barrier, which the other
+        // warps must also reach before they write s_o again; this warp's slice
+        // of s_v is rewritten only after its own reads above)
+        __syncwarp();
     }
     if (final_state) {
 #pragma unroll
